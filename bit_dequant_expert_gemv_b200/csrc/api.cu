@@ -1,0 +1,644 @@
+// api.cu — the C ABI declared in include/fmoe.h: argument validation, launch geometry, scratch
+// memory and CUDA-graph capture around the engine kernel (engine.cu) and the pack kernel.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "engine.h"
+#include "fmoe.h"
+
+extern "C" cudaError_t fmoe_engine_launch(const fmoe::Prog* P, const fmoe::Geo* G, int grid,
+                                          cudaStream_t stream);
+extern "C" cudaError_t fmoe_engine_configure(int max_smem);
+extern "C" cudaError_t fmoe_pack_launch(const float* w, int rows, int cols, int bits, void* dst,
+                                        int sms, cudaStream_t stream);
+
+using namespace fmoe;
+
+namespace {
+
+thread_local std::string g_err;
+thread_local uint64_t g_launches = 0;
+thread_local uint64_t g_wait_ns = 1000000000ull;
+thread_local int g_debug = 0;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define CK(call)                                        \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- per-device state
+struct DevState {
+  bool init = false;
+  int sms = 0;
+  int max_smem = 0;
+  int* err = nullptr;          // sticky device error word
+  cudaMemPool_t pool = nullptr;
+};
+std::mutex g_mu;
+DevState g_dev[64];
+
+int dev_state(DevState** out) {
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FMOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& d = g_dev[dev];
+  if (!d.init) {
+    CK(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    CK(cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    CK(cudaMalloc(&d.err, sizeof(int)));
+    CK(cudaMemset(d.err, 0, sizeof(int)));
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof props);
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    CK(cudaMemPoolCreate(&d.pool, &props));
+    uint64_t keep = 64ull << 20;  // keep up to 64 MiB of scratch cached between calls
+    CK(cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep));
+    CK(fmoe_engine_configure(d.max_smem));
+    d.init = true;
+  }
+  *out = &d;
+  return FMOE_OK;
+}
+
+int pad_slices(int s) {
+  if (s <= 32) {
+    int p = 1;
+    while (p < s) p <<= 1;
+    return p;
+  }
+  return (s + 31) / 32 * 32;
+}
+
+unsigned align_up(unsigned v, unsigned a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- validation and geometry
+int check_shape(int H, int I, int E, int K, int bits) {
+  if (bits != 2 && bits != 4) return fail(FMOE_ERR_INVALID, "bits must be 2 or 4 (got %d)", bits);
+  if (H <= 0 || I <= 0 || H % 64 || I % 64)
+    return fail(FMOE_ERR_INVALID, "hidden (%d) and inter (%d) must be positive multiples of 64", H, I);
+  if (E < 1 || K < 1 || K > E) return fail(FMOE_ERR_INVALID, "need 1 <= top_k (%d) <= n_experts (%d)", K, E);
+  if (H > 8192 || I > 8192) return fail(FMOE_ERR_UNSUPPORTED, "hidden/inter above 8192");
+  if (K > kMaxK) return fail(FMOE_ERR_UNSUPPORTED, "top_k above %d", kMaxK);
+  if (E > 4096) return fail(FMOE_ERR_UNSUPPORTED, "n_experts above 4096");
+  if ((long long)K * I > 8192) return fail(FMOE_ERR_UNSUPPORTED, "top_k * inter above 8192");
+  return FMOE_OK;
+}
+
+int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on, bool routed_on,
+             bool gate_on, int max_smem, Geo* G) {
+  memset(G, 0, sizeof *G);
+  G->H = H; G->I = I; G->E = E; G->K = K; G->bits = bits;
+  G->route_on = route_on; G->shared_on = shared_on; G->routed_on = routed_on;
+  G->gate_on = gate_on && route_on;
+  G->rc_h = (unsigned)H * bits / 8; G->rs_h = (unsigned)H / 16;
+  G->rc_i = (unsigned)I * bits / 8; G->rs_i = (unsigned)I / 16;
+  G->q_gu = (unsigned long long)I * (G->rc_h + G->rs_h);
+  G->q_dn = (unsigned long long)H * (G->rc_i + G->rs_i);
+  G->sl_h = H / 32; G->sp_h = pad_slices(G->sl_h); G->p_h = kConsumers / G->sp_h;
+  G->sl_i = I / 32; G->sp_i = pad_slices(G->sl_i); G->p_i = kConsumers / G->sp_i;
+  G->sl_d = K * G->sl_i; G->sp_d = pad_slices(G->sl_d); G->p_d = kConsumers / G->sp_d;
+  if (G->sp_h > kMaxSlices || G->sp_i > kMaxSlices || G->sp_d > kMaxSlices || G->p_h < 1 ||
+      G->p_i < 1 || G->p_d < 1)
+    return fail(FMOE_ERR_UNSUPPORTED, "row too wide for one CTA (H=%d I=%d K=%d)", H, I, K);
+  G->w_gu = G->p_h == 1 ? 8 : 4;
+  G->w_sd = 4;
+  G->w_rd = 4;
+  G->rcg = G->w_gu * G->p_h / 2;
+  G->rsd = 4 * G->p_i;
+  G->rrd = 4 * G->p_d;
+  G->nr = route_on ? E + (G->gate_on ? 1 : 0) : 0;
+  G->rr = std::max(1, std::min(32, 16384 / (4 * H)));
+  G->nb = (I + G->rcg - 1) / G->rcg;
+  G->n[P_ROUTER] = route_on ? (G->nr + G->rr - 1) / G->rr : 0;
+  G->n[P_SGU] = shared_on ? G->nb : 0;
+  G->n[P_SDN] = shared_on ? (H + G->rsd - 1) / G->rsd : 0;
+  G->n[P_RGU] = routed_on ? K * G->nb : 0;
+  G->n[P_RDN] = routed_on ? (H + G->rrd - 1) / G->rrd : 0;
+  G->off[0] = 0;
+  for (int p = 0; p < P_COUNT; ++p) G->off[p + 1] = G->off[p] + G->n[p];
+  if (G->off[P_COUNT] == 0) return fail(FMOE_ERR_INVALID, "nothing to compute");
+  unsigned stage = 0;
+  if (route_on) stage = std::max(stage, (unsigned)G->rr * 4u * H);
+  if (shared_on || routed_on) stage = std::max(stage, 2u * G->rcg * (G->rc_h + G->rs_h));
+  if (shared_on) stage = std::max(stage, (unsigned)G->rsd * (G->rc_i + G->rs_i));
+  if (routed_on) stage = std::max(stage, (unsigned)K * G->rrd * (G->rc_i + G->rs_i));
+  G->stage_bytes = align_up(stage, 128);
+  // fixed areas after the ring
+  unsigned o = 0;
+  auto take = [&](unsigned bytes) {
+    unsigned at = o;
+    o = align_up(o + bytes, 128);
+    return at;
+  };
+  G->o_xr = take(4u * H);
+  G->o_xg = take(4u * H);
+  G->o_sxg = take(4u * G->sl_h);
+  G->o_xs = take(4u * I);
+  G->o_sxs = take(4u * G->sl_i);
+  G->o_xd = take(4u * K * I);
+  G->o_sxd = take(4u * G->sl_d);
+  G->o_red = take(4u * 256 * 8);
+  G->o_misc = take(512);
+  const unsigned fixed = o;
+  const unsigned avail = (unsigned)max_smem - 1024;  // slack for alignment of the base
+  if (fixed + 2 * G->stage_bytes + 2 * 16 * 2 + 64 > avail)
+    return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for two stages");
+  int ns = (int)((avail - fixed - 256) / (G->stage_bytes + 20));
+  ns = std::min(ns, 16);
+  G->nstage = ns;
+  // final layout: ring | x areas (shifted) | barriers | meta
+  const unsigned ring = (unsigned)ns * G->stage_bytes;
+  G->o_ring = 0;
+  G->o_xr += ring; G->o_xg += ring; G->o_sxg += ring; G->o_xs += ring; G->o_sxs += ring;
+  G->o_xd += ring; G->o_sxd += ring; G->o_red += ring; G->o_misc += ring;
+  G->o_full = align_up(ring + fixed, 128);
+  G->o_empty = G->o_full + 8u * ns;
+  G->o_meta = G->o_empty + 8u * ns;
+  G->smem_bytes = align_up(G->o_meta + 4u * ns, 128);
+  if (G->smem_bytes > (unsigned)max_smem)
+    return fail(FMOE_ERR_UNSUPPORTED, "shared memory layout too large (%u)", G->smem_bytes);
+  return FMOE_OK;
+}
+
+int check_layer(const fmoe_layer_desc* L, const fmoe_layer_desc* L0) {
+  if (!L) return fail(FMOE_ERR_INVALID, "layer descriptor is NULL");
+  if (L0 && (L->hidden != L0->hidden || L->inter != L0->inter || L->n_experts != L0->n_experts ||
+             L->top_k != L0->top_k || L->bits != L0->bits))
+    return fail(FMOE_ERR_INVALID, "all layers must share hidden, inter, n_experts, top_k, bits");
+  int rc = check_shape(L->hidden, L->inter, L->n_experts, L->top_k, L->bits);
+  if (rc) return rc;
+  if (!L->experts || !L->router) return fail(FMOE_ERR_INVALID, "experts and router are required");
+  const size_t eb = fmoe_expert_bytes(L->hidden, L->inter, L->bits);
+  if (L->expert_stride < eb) return fail(FMOE_ERR_INVALID, "expert_stride (%zu) < expert bytes (%zu)", L->expert_stride, eb);
+  if (L->expert_stride % 16) return fail(FMOE_ERR_ALIGN, "expert_stride must be a multiple of 16");
+  if (!aligned16(L->experts) || !aligned16(L->router) || !aligned16(L->shared_expert) ||
+      !aligned16(L->shared_gate))
+    return fail(FMOE_ERR_ALIGN, "layer pointers must be 16-byte aligned");
+  return FMOE_OK;
+}
+
+// ---------------------------------------------------------------- scratch
+struct ScratchPlan {
+  size_t off_ctrl, off_normsq, zero_bytes, off_logits, off_sidx, off_sw, off_ssig, off_hs, off_hk,
+      off_hbuf, total;
+};
+
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+ScratchPlan plan_scratch(const Geo& G, int n_units) {
+  ScratchPlan s;
+  size_t o = 0;
+  s.off_ctrl = o; o = up256(o + 4 * C_WORDS);
+  s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
+  s.zero_bytes = o;
+  s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.nr, 1));
+  s.off_sidx = o; o = up256(o + 4 * 2 * (size_t)G.K);
+  s.off_sw = o; o = up256(o + 4 * 2 * (size_t)G.K);
+  s.off_ssig = o; o = up256(o + 4 * 2);
+  s.off_hs = o; o = up256(o + 4 * 2 * (size_t)G.I);
+  s.off_hk = o; o = up256(o + 4 * 2 * (size_t)G.K * G.I);
+  s.off_hbuf = o; o = up256(o + 4 * 2 * (size_t)G.H);
+  s.total = o;
+  return s;
+}
+
+void bind_scratch(Prog* P, const ScratchPlan& sp, uint8_t* base, int* err) {
+  P->s.ctrl = reinterpret_cast<unsigned*>(base + sp.off_ctrl);
+  P->s.normsq = reinterpret_cast<float*>(base + sp.off_normsq);
+  P->s.logits = reinterpret_cast<double*>(base + sp.off_logits);
+  P->s.sidx = reinterpret_cast<int*>(base + sp.off_sidx);
+  P->s.sw = reinterpret_cast<float*>(base + sp.off_sw);
+  P->s.ssig = reinterpret_cast<float*>(base + sp.off_ssig);
+  P->s.hs = reinterpret_cast<float*>(base + sp.off_hs);
+  P->s.hk = reinterpret_cast<float*>(base + sp.off_hk);
+  P->s.hbuf = reinterpret_cast<float*>(base + sp.off_hbuf);
+  P->s.err = err;
+}
+
+void fill_layers(Prog* P, const fmoe_layer_desc* layers, int n) {
+  for (int l = 0; l < n; ++l) {
+    P->layers[l].experts = static_cast<const uint8_t*>(layers[l].experts);
+    P->layers[l].expert_stride = layers[l].expert_stride;
+    P->layers[l].shared = static_cast<const uint8_t*>(layers[l].shared_expert);
+    P->layers[l].router = layers[l].router;
+    P->layers[l].gate = layers[l].shared_gate;
+  }
+}
+
+// Enqueue one engine run: zero the control words, launch.
+int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, int sms,
+                   cudaStream_t st) {
+  CK(cudaMemsetAsync(base, 0, sp.zero_bytes, st));
+  const long long total = (long long)P->n_units * G.off[P_COUNT];
+  const int grid = (int)std::min<long long>(sms, std::max<long long>(1, total));
+  cudaError_t e = fmoe_engine_launch(P, &G, grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "engine launch");
+  ++g_launches;
+  return FMOE_OK;
+}
+
+// Run a program with scratch taken from the library's stream-ordered pool.
+int run_pooled(Prog* P, const Geo& G, DevState* d, cudaStream_t st) {
+  const ScratchPlan sp = plan_scratch(G, P->n_units);
+  void* base = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&base, sp.total, d->pool, st);
+  if (e != cudaSuccess) return fail(FMOE_ERR_NOMEM, "scratch allocation: %s", cudaGetErrorString(e));
+  bind_scratch(P, sp, static_cast<uint8_t*>(base), d->err);
+  int rc = enqueue_engine(P, G, sp, static_cast<uint8_t*>(base), d->sms, st);
+  cudaError_t e2 = cudaFreeAsync(base, st);
+  if (rc) return rc;
+  if (e2 != cudaSuccess) return cuda_fail(e2, "scratch free");
+  return FMOE_OK;
+}
+
+void base_prog(Prog* P, int mode) {
+  memset(P, 0, sizeof *P);
+  P->mode = mode;
+  P->wait_ns = g_wait_ns;
+  P->debug = g_debug;
+}
+
+}  // namespace
+
+// =============================================================================================
+extern "C" {
+
+const char* fmoe_last_error(void) { return g_err.c_str(); }
+
+int fmoe_version(void) { return 10000; }
+
+void fmoe_set_wait_budget_ns(uint64_t ns) { g_wait_ns = ns < 1000 ? 1000 : ns; }
+
+void fmoe_set_fault_injection(int flags) { g_debug = flags; }
+
+uint64_t fmoe_launch_count(void) { return g_launches; }
+
+int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int bits, int flags,
+                           int max_smem, int64_t* out, int n_out) {
+  int rc = check_shape(hidden, inter, n_experts, top_k, bits);
+  if (rc) return rc;
+  Geo G;
+  if ((rc = make_geo(hidden, inter, n_experts, top_k, bits, flags & 1, flags & 2, flags & 4,
+                     flags & 8, max_smem, &G)))
+    return rc;
+  const int64_t v[] = {G.H, G.I, G.E, G.K, G.bits, G.route_on, G.shared_on, G.routed_on,
+                       G.gate_on, G.rc_h, G.rs_h, G.rc_i, G.rs_i, (int64_t)G.q_gu,
+                       (int64_t)G.q_dn, G.rr, G.rcg, G.rsd, G.rrd, G.nr, G.nb, G.n[0], G.n[1],
+                       G.n[2], G.n[3], G.n[4], G.off[0], G.off[1], G.off[2], G.off[3], G.off[4],
+                       G.off[5], G.sl_h, G.sp_h, G.p_h, G.sl_i, G.sp_i, G.p_i, G.sl_d, G.sp_d,
+                       G.p_d, G.w_gu, G.w_sd, G.w_rd, G.stage_bytes, G.nstage, G.o_ring,
+                       G.o_full, G.o_empty, G.o_meta, G.o_xr, G.o_xg, G.o_sxg, G.o_xs, G.o_sxs,
+                       G.o_xd, G.o_sxd, G.o_red, G.o_misc, G.smem_bytes};
+  const int n = (int)(sizeof v / sizeof v[0]);
+  for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
+  return n < n_out ? n : n_out;
+}
+
+int fmoe_sync_status(void* stream) {
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  CK(cudaMemcpy(&v, d->err, sizeof v, cudaMemcpyDeviceToHost));
+  if (v == 0) return FMOE_OK;
+  CK(cudaMemset(d->err, 0, sizeof(int)));
+  static const char* what[] = {"", "waiting for a weight stage", "waiting for a free stage",
+                               "waiting for the routing decision", "waiting for a dependency",
+                               "draining copies"};
+  return fail(FMOE_ERR_TIMEOUT, "a device-side wait ran out of budget (%s)",
+              v > 0 && v < 6 ? what[v] : "?");
+}
+
+size_t fmoe_qmat_bytes(int rows, int cols, int bits) {
+  if (rows <= 0 || cols <= 0 || rows % 64 || cols % 64 || (bits != 2 && bits != 4)) return 0;
+  const size_t n = (size_t)rows * (size_t)cols;
+  return n * (size_t)bits / 8 + n / 16;
+}
+
+size_t fmoe_expert_bytes(int hidden, int inter, int bits) {
+  const size_t a = fmoe_qmat_bytes(inter, hidden, bits), b = fmoe_qmat_bytes(hidden, inter, bits);
+  if (!a || !b) return 0;
+  return 2 * a + b;
+}
+
+int fmoe_pack(const float* w, int rows, int cols, int bits, void* dst, void* stream) {
+  if (bits != 2 && bits != 4) return fail(FMOE_ERR_INVALID, "bits must be 2 or 4 (got %d)", bits);
+  if (rows <= 0 || cols <= 0 || rows % 64 || cols % 64 || rows > (1 << 20) || cols > (1 << 16))
+    return fail(FMOE_ERR_INVALID, "rows (%d) and cols (%d) must be positive multiples of 64", rows, cols);
+  if (!w || !dst) return fail(FMOE_ERR_INVALID, "NULL pointer");
+  if (!aligned16(w) || !aligned16(dst)) return fail(FMOE_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const char* wb = reinterpret_cast<const char*>(w);
+  const char* db = static_cast<const char*>(dst);
+  if (wb < db + fmoe_qmat_bytes(rows, cols, bits) && db < wb + (size_t)rows * cols * 4)
+    return fail(FMOE_ERR_INVALID, "w and dst overlap");
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  cudaError_t e = fmoe_pack_launch(w, rows, cols, bits, dst, d->sms, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  ++g_launches;
+  return FMOE_OK;
+}
+
+int fmoe_pack_q4(const float* w, int rows, int cols, void* dst, void* stream) {
+  return fmoe_pack(w, rows, cols, 4, dst, stream);
+}
+
+int fmoe_pack_q2(const float* w, int rows, int cols, void* dst, void* stream) {
+  return fmoe_pack(w, rows, cols, 2, dst, stream);
+}
+
+int fmoe_route(const float* x, const float* router, const float* logit_bias, int hidden,
+               int n_experts, int top_k, int32_t* idx, float* weight, void* stream) {
+  int rc = check_shape(hidden, 64, n_experts, top_k, 4);
+  if (rc) return rc;
+  if (!x || !router || !idx || !weight) return fail(FMOE_ERR_INVALID, "NULL pointer");
+  if (!aligned16(x) || !aligned16(router))
+    return fail(FMOE_ERR_ALIGN, "x and router must be 16-byte aligned");
+  DevState* d;
+  if ((rc = dev_state(&d))) return rc;
+  Geo G;
+  if ((rc = make_geo(hidden, 64, n_experts, top_k, 4, true, false, false, false, d->max_smem, &G)))
+    return rc;
+  Prog P;
+  base_prog(&P, MODE_SEQ);
+  P.n_units = 1; P.n_layers = 1; P.n_tokens = 1;
+  P.x = x; P.bias = logit_bias; P.idx_out = idx; P.w_out = weight;
+  P.out = nullptr;
+  P.layers[0].router = router;
+  return run_pooled(&P, G, d, static_cast<cudaStream_t>(stream));
+}
+
+int fmoe_expert_gemv(const void* expert, int hidden, int inter, int bits, const float* x,
+                     float* y, void* stream) {
+  int rc = check_shape(hidden, inter, 1, 1, bits);
+  if (rc) return rc;
+  if (!expert || !x || !y) return fail(FMOE_ERR_INVALID, "NULL pointer");
+  if (!aligned16(expert) || !aligned16(x) || !aligned16(y))
+    return fail(FMOE_ERR_ALIGN, "pointers must be 16-byte aligned");
+  if (x == y) return fail(FMOE_ERR_INVALID, "x and y must not alias");
+  DevState* d;
+  if ((rc = dev_state(&d))) return rc;
+  Geo G;
+  if ((rc = make_geo(hidden, inter, 1, 1, bits, false, true, false, false, d->max_smem, &G)))
+    return rc;
+  Prog P;
+  base_prog(&P, MODE_SEQ);
+  P.n_units = 1; P.n_layers = 1; P.n_tokens = 1;
+  P.x = x; P.out = y;
+  P.layers[0].shared = static_cast<const uint8_t*>(expert);
+  return run_pooled(&P, G, d, static_cast<cudaStream_t>(stream));
+}
+
+static int prep_layers(const fmoe_layer_desc* layers, int n_layers, DevState* d, Geo* G) {
+  if (!layers || n_layers < 1 || n_layers > kMaxLayers)
+    return fail(FMOE_ERR_INVALID, "need 1 <= n_layers <= %d", kMaxLayers);
+  int rc;
+  for (int l = 0; l < n_layers; ++l)
+    if ((rc = check_layer(&layers[l], l ? &layers[0] : nullptr))) return rc;
+  bool shared = layers[0].shared_expert != nullptr, gate = layers[0].shared_gate != nullptr;
+  for (int l = 1; l < n_layers; ++l)
+    if ((layers[l].shared_expert != nullptr) != shared || (layers[l].shared_gate != nullptr) != gate)
+      return fail(FMOE_ERR_INVALID, "all layers must agree on having a shared expert / gate");
+  const fmoe_layer_desc& L = layers[0];
+  return make_geo(L.hidden, L.inter, L.n_experts, L.top_k, L.bits, true, shared, true,
+                  gate && shared, d->max_smem, G);
+}
+
+int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float* x,
+                       const float* residual, int n_tokens, const float* logit_bias, float* out,
+                       int32_t* idx_out, float* w_out, void* stream) {
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  Geo G;
+  if ((rc = prep_layers(layers, n_layers, d, &G))) return rc;
+  if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
+  if ((long long)n_tokens * G.off[P_COUNT] > 0x7ffffff0ll) return fail(FMOE_ERR_UNSUPPORTED, "too many tokens");
+  if (!x || !out) return fail(FMOE_ERR_INVALID, "x and out are required");
+  if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
+    return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
+  if (x == out) return fail(FMOE_ERR_INVALID, "x must not alias out");
+  Prog P;
+  base_prog(&P, MODE_SEQ);
+  P.n_units = n_tokens; P.n_layers = n_layers; P.n_tokens = n_tokens;
+  P.x = x; P.res = residual; P.out = out; P.bias = logit_bias; P.idx_out = idx_out; P.w_out = w_out;
+  fill_layers(&P, layers, n_layers);
+  return run_pooled(&P, G, d, static_cast<cudaStream_t>(stream));
+}
+
+int fmoe_moe_layer_seq_host(const fmoe_layer_desc* layers, int n_layers, const float* x_host,
+                            const float* residual_host, int n_tokens,
+                            const float* logit_bias_host, float* out_host, int32_t* idx_host,
+                            float* w_host, void* stream) {
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  Geo G;
+  if ((rc = prep_layers(layers, n_layers, d, &G))) return rc;
+  if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
+  if (!x_host || !out_host) return fail(FMOE_ERR_INVALID, "x_host and out_host are required");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t T = (size_t)n_tokens, H = (size_t)G.H, E = (size_t)G.E, K = (size_t)G.K;
+  size_t o = 0;
+  const size_t ox = o; o = up256(o + T * H * 4);
+  const size_t orr = o; o = up256(o + (residual_host ? T * H * 4 : 0));
+  const size_t ob = o; o = up256(o + (logit_bias_host ? T * E * 4 : 0));
+  const size_t oo = o; o = up256(o + T * H * 4);
+  const size_t oi = o; o = up256(o + T * K * 4);
+  const size_t ow = o; o = up256(o + T * K * 4);
+  void* dev = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&dev, o, d->pool, st);
+  if (e != cudaSuccess) return fail(FMOE_ERR_NOMEM, "staging allocation: %s", cudaGetErrorString(e));
+  uint8_t* b = static_cast<uint8_t*>(dev);
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    return n ? cudaMemcpyAsync(b + off, src, n, cudaMemcpyHostToDevice, st) : cudaSuccess;
+  };
+  if ((e = h2d(ox, x_host, T * H * 4)) != cudaSuccess ||
+      (residual_host && (e = h2d(orr, residual_host, T * H * 4)) != cudaSuccess) ||
+      (logit_bias_host && (e = h2d(ob, logit_bias_host, T * E * 4)) != cudaSuccess)) {
+    cudaFreeAsync(dev, st);
+    return cuda_fail(e, "host->device copy");
+  }
+  rc = fmoe_moe_layer_seq(layers, n_layers, reinterpret_cast<float*>(b + ox),
+                          residual_host ? reinterpret_cast<float*>(b + orr) : nullptr, n_tokens,
+                          logit_bias_host ? reinterpret_cast<float*>(b + ob) : nullptr,
+                          reinterpret_cast<float*>(b + oo), idx_host ? reinterpret_cast<int32_t*>(b + oi) : nullptr,
+                          w_host ? reinterpret_cast<float*>(b + ow) : nullptr, stream);
+  if (rc == FMOE_OK) {
+    if ((e = cudaMemcpyAsync(out_host, b + oo, T * H * 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (idx_host && (e = cudaMemcpyAsync(idx_host, b + oi, T * K * 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess) ||
+        (w_host && (e = cudaMemcpyAsync(w_host, b + ow, T * K * 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess))
+      rc = cuda_fail(e, "device->host copy");
+  }
+  cudaFreeAsync(dev, st);
+  return rc;
+}
+
+int fmoe_moe_layer(const fmoe_layer_desc* layer, const float* x, const float* residual,
+                   const float* logit_bias, float* out, int32_t* idx_out, float* w_out,
+                   void* stream) {
+  return fmoe_moe_layer_seq(layer, 1, x, residual, 1, logit_bias, out, idx_out, w_out, stream);
+}
+
+static int stack_prog(const fmoe_layer_desc* layers, int n_layers, const float* h_in,
+                      int n_tokens, const float* logit_bias, float eps, float* h_out,
+                      int32_t* idx_trace, float* h_trace, DevState* d, Geo* G, Prog* P) {
+  int rc = prep_layers(layers, n_layers, d, G);
+  if (rc) return rc;
+  if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
+  if ((long long)n_tokens * n_layers * G->off[P_COUNT] > 0x7ffffff0ll)
+    return fail(FMOE_ERR_UNSUPPORTED, "too many tokens x layers for one launch");
+  if (!h_in || !h_out) return fail(FMOE_ERR_INVALID, "h_in and h_out are required");
+  if (!aligned16(h_in) || !aligned16(h_out) || !aligned16(h_trace))
+    return fail(FMOE_ERR_ALIGN, "h_in, h_out, h_trace must be 16-byte aligned");
+  if (h_in == h_out) return fail(FMOE_ERR_INVALID, "h_out must not alias h_in");
+  if (!(eps >= 0.f)) return fail(FMOE_ERR_INVALID, "eps must be >= 0");
+  base_prog(P, MODE_STACK);
+  P->n_units = n_tokens * n_layers; P->n_layers = n_layers; P->n_tokens = n_tokens;
+  P->x = h_in; P->out = h_out; P->bias = logit_bias; P->idx_out = idx_trace; P->h_trace = h_trace;
+  P->eps = eps;
+  fill_layers(P, layers, n_layers);
+  return FMOE_OK;
+}
+
+int fmoe_moe_stack(const fmoe_layer_desc* layers, int n_layers, const float* h_in, int n_tokens,
+                   const float* logit_bias, float eps, float* h_out, int32_t* idx_trace,
+                   float* h_trace, void* stream) {
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  Geo G;
+  Prog P;
+  if ((rc = stack_prog(layers, n_layers, h_in, n_tokens, logit_bias, eps, h_out, idx_trace,
+                       h_trace, d, &G, &P)))
+    return rc;
+  return run_pooled(&P, G, d, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+struct fmoe_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  void* scratch = nullptr;
+  int kernels = 0;
+};
+
+extern "C" {
+
+int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const float* h_in,
+                            int n_tokens, const float* logit_bias, float eps, float* h_out,
+                            int32_t* idx_trace, float* h_trace, int tokens_per_launch,
+                            fmoe_graph** graph) {
+  if (!graph) return fail(FMOE_ERR_INVALID, "graph out-pointer is NULL");
+  *graph = nullptr;
+  DevState* d;
+  int rc = dev_state(&d);
+  if (rc) return rc;
+  Geo G;
+  Prog P;
+  if ((rc = stack_prog(layers, n_layers, h_in, n_tokens, logit_bias, eps, h_out, idx_trace,
+                       h_trace, d, &G, &P)))
+    return rc;
+  if (tokens_per_launch <= 0 || tokens_per_launch > n_tokens) tokens_per_launch = n_tokens;
+  const int H = G.H, E = G.E, K = G.K, L = n_layers;
+  const int units_per_launch = tokens_per_launch * L;
+  const ScratchPlan sp = plan_scratch(G, units_per_launch);
+  fmoe_graph* g = new fmoe_graph();
+  cudaError_t e = cudaMalloc(&g->scratch, sp.total);
+  if (e != cudaSuccess) {
+    delete g;
+    return fail(FMOE_ERR_NOMEM, "graph scratch: %s", cudaGetErrorString(e));
+  }
+  cudaStream_t cs;
+  if ((e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking)) != cudaSuccess) {
+    cudaFree(g->scratch);
+    delete g;
+    return cuda_fail(e, "capture stream");
+  }
+  const uint64_t launches_before = g_launches;
+  e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (e == cudaSuccess) {
+    for (int t0 = 0; t0 < n_tokens && rc == FMOE_OK; t0 += tokens_per_launch) {
+      const int nt = std::min(tokens_per_launch, n_tokens - t0);
+      Prog Q = P;
+      Q.n_tokens = nt;
+      Q.n_units = nt * L;
+      Q.x = h_in + (size_t)t0 * H;
+      Q.out = h_out + (size_t)t0 * H;
+      Q.bias = logit_bias ? logit_bias + (size_t)t0 * L * E : nullptr;
+      Q.idx_out = idx_trace ? idx_trace + (size_t)t0 * L * K : nullptr;
+      Q.h_trace = h_trace ? h_trace + (size_t)t0 * L * H : nullptr;
+      bind_scratch(&Q, sp, static_cast<uint8_t*>(g->scratch), d->err);
+      rc = enqueue_engine(&Q, G, sp, static_cast<uint8_t*>(g->scratch), d->sms, cs);
+    }
+    cudaError_t e2 = cudaStreamEndCapture(cs, &g->graph);
+    if (rc == FMOE_OK && e2 != cudaSuccess) rc = cuda_fail(e2, "end capture");
+  } else {
+    rc = cuda_fail(e, "begin capture");
+  }
+  cudaStreamDestroy(cs);
+  g->kernels = (int)(g_launches - launches_before);
+  g_launches = launches_before;
+  if (rc == FMOE_OK) {
+    e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+    if (e != cudaSuccess) rc = cuda_fail(e, "graph instantiate");
+  }
+  if (rc != FMOE_OK) {
+    if (g->graph) cudaGraphDestroy(g->graph);
+    cudaFree(g->scratch);
+    delete g;
+    return rc;
+  }
+  *graph = g;
+  return FMOE_OK;
+}
+
+int fmoe_stack_graph_launch(fmoe_graph* g, void* stream) {
+  if (!g || !g->exec) return fail(FMOE_ERR_INVALID, "graph is NULL");
+  cudaError_t e = cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "graph launch");
+  g_launches += (uint64_t)g->kernels;
+  return FMOE_OK;
+}
+
+int fmoe_stack_graph_destroy(fmoe_graph* g) {
+  if (!g) return FMOE_OK;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  if (g->scratch) cudaFree(g->scratch);
+  delete g;
+  return FMOE_OK;
+}
+
+}  // extern "C"

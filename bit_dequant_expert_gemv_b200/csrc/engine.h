@@ -1,0 +1,105 @@
+// engine.h — host/device description of one launch of the MoE engine kernel.
+//
+// A launch runs a sequence of "units"; a unit is one MoE layer applied to one token. The work
+// of a unit is cut into chunks, listed in dependency order by phase:
+//   P_ROUTER   router rows (fp32, binary64 accumulation) + the shared-gate row; the CTA that
+//              completes the last router chunk selects the top-K experts
+//   P_SGU      shared expert gate/up rows + SwiGLU            (needs x)
+//   P_SDN      shared expert down rows + residual             (needs the shared h and sigma)
+//   P_RGU      routed experts gate/up rows + SwiGLU           (needs the routing decision)
+//   P_RDN      routed experts down rows + weighted combine    (needs all routed h)
+// Chunks are claimed through one global counter in that order, so every wait a chunk makes is
+// on chunks with smaller indices: the schedule cannot deadlock whatever the residency.
+#pragma once
+#include <stdint.h>
+
+namespace fmoe {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;    // 256 consumer threads
+constexpr int kThreads = kConsumers + 32;          // + one producer warp
+constexpr int kMaxLayers = 128;
+constexpr int kMaxK = 8;
+constexpr int kMaxSlices = 256;                    // 32-column slices per (virtual) row
+constexpr int kSliceCols = 32;
+
+enum Phase { P_ROUTER = 0, P_SGU = 1, P_SDN = 2, P_RGU = 3, P_RDN = 4, P_COUNT = 5 };
+
+// control words (uint32, zeroed before every launch)
+enum Ctrl {
+  C_NEXT = 0,          // next chunk to claim
+  C_CNT = 1,           // C_CNT + phase: chunks of that phase completed (monotonic over units)
+  C_ROUTE = 8,         // number of units whose routing decision is published
+  C_WORDS = 16
+};
+
+enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
+
+struct LayerW {
+  const uint8_t* experts;
+  unsigned long long expert_stride;
+  const uint8_t* shared;       // nullable
+  const float* router;         // [E x H]
+  const float* gate;           // nullable [H]
+};
+
+struct Geo {
+  int H, I, E, K, bits;
+  int route_on, shared_on, routed_on, gate_on;
+  // bytes per row
+  unsigned rc_h, rs_h, rc_i, rs_i;
+  unsigned long long q_gu, q_dn;  // bytes of an I x H (gate/up) and an H x I (down) packed matrix
+  // rows per chunk
+  int rr, rcg, rsd, rrd;
+  int nr;                      // router rows: E + gate_on
+  int nb;                      // gate/up chunks per expert
+  int n[P_COUNT];
+  int off[P_COUNT + 1];        // off[P_COUNT] = chunks per unit
+  // thread mapping: slices of 32 columns, padded per virtual row
+  int sl_h, sp_h, p_h;         // H-wide rows (gate/up)
+  int sl_i, sp_i, p_i;         // I-wide rows (shared down)
+  int sl_d, sp_d, p_d;         // K*I-wide virtual rows (routed down)
+  int w_gu, w_sd, w_rd;        // waves per chunk
+  // shared memory carve-up (byte offsets from the dynamic smem base)
+  unsigned stage_bytes;
+  int nstage;
+  unsigned o_ring, o_full, o_empty, o_meta, o_xr, o_xg, o_sxg, o_xs, o_sxs, o_xd, o_sxd, o_red,
+      o_rows, o_misc;
+  unsigned smem_bytes;
+};
+
+struct Scratch {
+  unsigned* ctrl;        // C_WORDS
+  int* err;              // sticky per-device error word
+  double* logits;        // [2][nr]
+  int* sidx;             // [2][K]
+  float* sw;             // [2][K]
+  float* ssig;           // [2]
+  float* hs;             // [2][I]
+  float* hk;             // [2][K][I]
+  float* normsq;         // [n_units]
+  float* hbuf;           // [2][H]
+};
+
+struct Prog {
+  int mode;
+  int n_units, n_layers, n_tokens;
+  const float* x;        // SEQ: [T x H] inputs; STACK: h_in
+  const float* res;      // SEQ: nullable [T x H]
+  float* out;            // SEQ: [T x H]; STACK: h_out
+  const float* bias;     // SEQ: [T x E]; STACK: [T x L x E]; nullable
+  int* idx_out;          // SEQ: [T x K]; STACK: [T x L x K]; nullable
+  float* w_out;          // SEQ: [T x K]; nullable
+  float* h_trace;        // STACK: [T x L x H] layer inputs before the norm; nullable
+  float eps;
+  unsigned long long wait_ns;
+  int debug;             // bit 0: the routing decision is never published (timeout test)
+  Scratch s;
+  LayerW layers[kMaxLayers];
+};
+
+// error codes written to Scratch::err (first one wins)
+enum DevErr { DE_NONE = 0, DE_TIMEOUT_FULL = 1, DE_TIMEOUT_EMPTY = 2, DE_TIMEOUT_ROUTE = 3,
+              DE_TIMEOUT_DEP = 4, DE_TIMEOUT_DRAIN = 5 };
+
+}  // namespace fmoe

@@ -95,6 +95,12 @@ int fmoe_sync_status(void* stream);
  * calling host thread, in nanoseconds (default 1e9 = 1 s; values < 1000 are clamped). */
 void fmoe_set_wait_budget_ns(uint64_t ns);
 
+/* Test hook: bit 0 makes every kernel launched afterwards on the calling host thread compute
+ * but never publish its routing decision, so every wait that depends on it runs out of its
+ * budget and the launch ends with FMOE_ERR_TIMEOUT (a host-made failure for testing the
+ * timeout path; nothing faults). 0 restores normal operation. */
+void fmoe_set_fault_injection(int flags);
+
 /* ---------------------------------------------------------------------------------------
  * Sizes (host only; no CUDA call). Return 0 for an illegal (rows, cols, bits).
  * --------------------------------------------------------------------------------------- */
@@ -183,6 +189,18 @@ int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float*
                        const float* residual, int n_tokens, const float* logit_bias,
                        float* out, int32_t* idx_out, float* w_out, void* stream);
 
+/* Same as fmoe_moe_layer_seq with the token data in HOST memory: x_host, residual_host
+ * (nullable), logit_bias_host (nullable), out_host, idx_host and w_host (both nullable) are
+ * host pointers (page-locked for the copies to be asynchronous). The call stages them
+ * through library-owned device memory on `stream` with one cudaMemcpyAsync per buffer:
+ * inputs host->device, the launch, outputs device->host. Host buffers must stay valid and
+ * unmodified until `stream` has completed the call. Layer descriptors are device memory as
+ * usual. */
+int fmoe_moe_layer_seq_host(const fmoe_layer_desc* layers, int n_layers, const float* x_host,
+                            const float* residual_host, int n_tokens,
+                            const float* logit_bias_host, float* out_host, int32_t* idx_host,
+                            float* w_host, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * MoE-only decode stack: n_tokens tokens, each through n_layers layers in order, token by
  * token ([JA-O] "遅延GPUエキスパート計算": the combine + residual + norm output feeds the next
@@ -192,12 +210,13 @@ int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float*
  *   h_{l+1} = MoE layer l (x_l, residual = h_l)
  *   h_out[t] = h_L
  * logit_bias: nullable [T x L x E]. idx_trace: nullable [T x L x K] int32 (chosen experts).
- * x_trace: nullable [T x L x H] fp32 (the normalised x_l, for teacher-forced checking).
+ * h_trace: nullable [T x L x H] fp32: the input h_l of every layer before its RMSNorm (h_0 =
+ * h_in), for teacher-forced checking of single layers.
  * 1 <= n_layers <= 128; all layers share H, I, E, K, bits. h_out must not alias h_in.
  * --------------------------------------------------------------------------------------- */
 int fmoe_moe_stack(const fmoe_layer_desc* layers, int n_layers, const float* h_in,
                    int n_tokens, const float* logit_bias, float eps, float* h_out,
-                   int32_t* idx_trace, float* x_trace, void* stream);
+                   int32_t* idx_trace, float* h_trace, void* stream);
 
 /* Same computation as fmoe_moe_stack, captured once into a CUDA graph that owns its scratch
  * memory; fmoe_stack_graph_launch replays it on `stream` (same buffers every replay).
@@ -207,10 +226,23 @@ int fmoe_moe_stack(const fmoe_layer_desc* layers, int n_layers, const float* h_i
 typedef struct fmoe_graph fmoe_graph;
 int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const float* h_in,
                             int n_tokens, const float* logit_bias, float eps, float* h_out,
-                            int32_t* idx_trace, float* x_trace, int tokens_per_launch,
+                            int32_t* idx_trace, float* h_trace, int tokens_per_launch,
                             fmoe_graph** graph);
 int fmoe_stack_graph_launch(fmoe_graph* graph, void* stream);
 int fmoe_stack_graph_destroy(fmoe_graph* graph);
+
+/* Launch geometry of the engine kernel for a shape (host only; no CUDA call). flags: bit 0
+ * router, bit 1 shared expert, bit 2 routed experts, bit 3 shared-expert gate. Writes up to
+ * n_out int64 values in the order documented in FMOE_GEOMETRY_FIELDS and returns how many
+ * were written, or a negative status for an unsupported shape. For checking the launch
+ * layout against buffer bounds on a machine without a GPU. */
+#define FMOE_GEOMETRY_FIELDS                                                                  \
+    "H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu q_dn rr rcg " \
+    "rsd rrd nr nb n0 n1 n2 n3 n4 off0 off1 off2 off3 off4 off5 sl_h sp_h p_h sl_i sp_i p_i " \
+    "sl_d sp_d p_d w_gu w_sd w_rd stage_bytes nstage o_ring o_full o_empty o_meta o_xr o_xg " \
+    "o_sxg o_xs o_sxs o_xd o_sxd o_red o_misc smem_bytes"
+int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int bits, int flags,
+                           int max_smem, int64_t* out, int n_out);
 
 /* Number of kernel launches of this library enqueued on the calling host thread so far
  * (graph replays count the kernels inside the graph). For accounting in benchmarks. */
