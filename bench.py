@@ -42,6 +42,8 @@ def parse():
                     choices=["full_q4", "full_q4_natural", "full_q2", "stack_q4_uniform",
                              "stack_q4_skewed", "stack_q2"])
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0 = workload's)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the number of routed experts (small cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -224,6 +226,9 @@ def run_ours(args):
     fmoe.build()
 
     wl = synth.WORKLOADS[args.workload]
+    if args.experts:
+        import dataclasses
+        wl = dataclasses.replace(wl, E=args.experts, name=f"{wl.name}_E{args.experts}")
     stack = wl.layers > 1
     T = args.tokens or wl.tokens
     # rank r runs its own stream of tokens (different x), same weights

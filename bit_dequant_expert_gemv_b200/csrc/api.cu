@@ -165,7 +165,15 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   G->o_sxs = take(4u * G->sl_i);
   G->o_xd = take(4u * K * I);
   G->o_sxd = take(4u * G->sl_d);
-  G->o_red = take(4u * 256 * 8);
+  // reduction slot: per-warp (or per-segment) row partials, kMaxW per segment; router rows
+  // as binary64 partials of 8 warps x rr rows; then one prefetched base per output row
+  auto nseg = [](int sp) { return sp >= 32 ? kConsumerWarps : kConsumers / sp; };
+  const int part = std::max(std::max(nseg(G->sp_h), std::max(nseg(G->sp_i), nseg(G->sp_d))) * 8,
+                            2 * kConsumerWarps * G->rr);
+  G->red_part = (part + 31) / 32 * 32;
+  G->box_floats = G->red_part + (std::max(G->rsd, G->rrd) + 31) / 32 * 32;
+  G->o_red = take(16);
+  G->o_box = take(4u * kBoxes * G->box_floats);
   G->o_misc = take(512);
   const unsigned fixed = o;
   const unsigned avail = (unsigned)max_smem - 1024;  // slack for alignment of the base
@@ -178,7 +186,7 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   const unsigned ring = (unsigned)ns * G->stage_bytes;
   G->o_ring = 0;
   G->o_xr += ring; G->o_xg += ring; G->o_sxg += ring; G->o_xs += ring; G->o_sxs += ring;
-  G->o_xd += ring; G->o_sxd += ring; G->o_red += ring; G->o_misc += ring;
+  G->o_xd += ring; G->o_sxd += ring; G->o_red += ring; G->o_misc += ring; G->o_box += ring;
   G->o_full = align_up(ring + fixed, 128);
   G->o_empty = G->o_full + 8u * ns;
   G->o_meta = G->o_empty + 8u * ns;
@@ -207,22 +215,19 @@ int check_layer(const fmoe_layer_desc* L, const fmoe_layer_desc* L0) {
 
 // ---------------------------------------------------------------- scratch
 struct ScratchPlan {
-  size_t off_ctrl, off_normsq, zero_bytes, off_logits, off_sidx, off_sw, off_ssig, off_hs, off_hk,
-      off_hbuf, total;
+  size_t off_ctrl, off_flags, off_normsq, zero_bytes, off_logits, off_hs, off_hk, off_hbuf, total;
 };
 
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
-ScratchPlan plan_scratch(const Geo& G, int n_units) {
+ScratchPlan plan_scratch(const Geo& G, int n_units, int max_grid) {
   ScratchPlan s;
   size_t o = 0;
   s.off_ctrl = o; o = up256(o + 4 * C_WORDS);
+  s.off_flags = o; o = up256(o + 4 * (size_t)F_WORDS * max_grid);
   s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
   s.zero_bytes = o;
   s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.nr, 1));
-  s.off_sidx = o; o = up256(o + 4 * 2 * (size_t)G.K);
-  s.off_sw = o; o = up256(o + 4 * 2 * (size_t)G.K);
-  s.off_ssig = o; o = up256(o + 4 * 2);
   s.off_hs = o; o = up256(o + 4 * 2 * (size_t)G.I);
   s.off_hk = o; o = up256(o + 4 * 2 * (size_t)G.K * G.I);
   s.off_hbuf = o; o = up256(o + 4 * 2 * (size_t)G.H);
@@ -232,11 +237,9 @@ ScratchPlan plan_scratch(const Geo& G, int n_units) {
 
 void bind_scratch(Prog* P, const ScratchPlan& sp, uint8_t* base, int* err) {
   P->s.ctrl = reinterpret_cast<unsigned*>(base + sp.off_ctrl);
+  P->s.flags = reinterpret_cast<unsigned*>(base + sp.off_flags);
   P->s.normsq = reinterpret_cast<float*>(base + sp.off_normsq);
   P->s.logits = reinterpret_cast<double*>(base + sp.off_logits);
-  P->s.sidx = reinterpret_cast<int*>(base + sp.off_sidx);
-  P->s.sw = reinterpret_cast<float*>(base + sp.off_sw);
-  P->s.ssig = reinterpret_cast<float*>(base + sp.off_ssig);
   P->s.hs = reinterpret_cast<float*>(base + sp.off_hs);
   P->s.hk = reinterpret_cast<float*>(base + sp.off_hk);
   P->s.hbuf = reinterpret_cast<float*>(base + sp.off_hbuf);
@@ -267,7 +270,7 @@ int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, 
 
 // Run a program with scratch taken from the library's stream-ordered pool.
 int run_pooled(Prog* P, const Geo& G, DevState* d, cudaStream_t st) {
-  const ScratchPlan sp = plan_scratch(G, P->n_units);
+  const ScratchPlan sp = plan_scratch(G, P->n_units, d->sms);
   void* base = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&base, sp.total, d->pool, st);
   if (e != cudaSuccess) return fail(FMOE_ERR_NOMEM, "scratch allocation: %s", cudaGetErrorString(e));
@@ -316,7 +319,8 @@ int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int 
                        G.off[5], G.sl_h, G.sp_h, G.p_h, G.sl_i, G.sp_i, G.p_i, G.sl_d, G.sp_d,
                        G.p_d, G.w_gu, G.w_sd, G.w_rd, G.stage_bytes, G.nstage, G.o_ring,
                        G.o_full, G.o_empty, G.o_meta, G.o_xr, G.o_xg, G.o_sxg, G.o_xs, G.o_sxs,
-                       G.o_xd, G.o_sxd, G.o_red, G.o_misc, G.smem_bytes};
+                       G.o_xd, G.o_sxd, G.o_red, G.o_misc, G.smem_bytes, G.o_box,
+                       G.box_floats, G.red_part};
   const int n = (int)(sizeof v / sizeof v[0]);
   for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
   return n < n_out ? n : n_out;
@@ -573,7 +577,7 @@ int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const f
   if (tokens_per_launch <= 0 || tokens_per_launch > n_tokens) tokens_per_launch = n_tokens;
   const int H = G.H, E = G.E, K = G.K, L = n_layers;
   const int units_per_launch = tokens_per_launch * L;
-  const ScratchPlan sp = plan_scratch(G, units_per_launch);
+  const ScratchPlan sp = plan_scratch(G, units_per_launch, d->sms);
   fmoe_graph* g = new fmoe_graph();
   cudaError_t e = cudaMalloc(&g->scratch, sp.total);
   if (e != cudaSuccess) {

@@ -2,14 +2,16 @@
 //
 // A launch runs a sequence of "units"; a unit is one MoE layer applied to one token. The work
 // of a unit is cut into chunks, listed in dependency order by phase:
-//   P_ROUTER   router rows (fp32, binary64 accumulation) + the shared-gate row; the CTA that
-//              completes the last router chunk selects the top-K experts
+//   P_ROUTER   router rows (fp32, binary64 accumulation) + the shared-gate row; the CTA whose
+//              completion brings the router count to its target selects the top-K experts
 //   P_SGU      shared expert gate/up rows + SwiGLU            (needs x)
 //   P_SDN      shared expert down rows + residual             (needs the shared h and sigma)
 //   P_RGU      routed experts gate/up rows + SwiGLU           (needs the routing decision)
 //   P_RDN      routed experts down rows + weighted combine    (needs all routed h)
-// Chunks are claimed through one global counter in that order, so every wait a chunk makes is
-// on chunks with smaller indices: the schedule cannot deadlock whatever the residency.
+// Chunk g of the launch (g = unit * chunks_per_unit + index) belongs to CTA g mod gridDim, and
+// every CTA works through its chunks in increasing g; every wait a chunk makes is on chunks with
+// smaller g, so with all CTAs resident (one per SM) the schedule cannot deadlock, and every wait
+// is bounded in time in any case.
 #pragma once
 #include <stdint.h>
 
@@ -17,20 +19,22 @@ namespace fmoe {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;    // 256 consumer threads
-constexpr int kThreads = kConsumers + 32;          // + one producer warp
+constexpr int kThreads = kConsumers + 64;          // + one producer warp + one signal warp
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
 constexpr int kMaxSlices = 256;                    // 32-column slices per (virtual) row
 constexpr int kSliceCols = 32;
+constexpr int kBoxes = 4;                          // outbox depth (chunks)
 
 enum Phase { P_ROUTER = 0, P_SGU = 1, P_SDN = 2, P_RGU = 3, P_RDN = 4, P_COUNT = 5 };
 
-// control words (uint32, zeroed before every launch)
+// Control words (uint32, zeroed before every launch). Phase counters take one atomic per CTA
+// per run of chunks; the CTA whose atomic completes a phase of a unit writes "phase p of unit
+// u is complete" into every CTA's own flag line, and waiters poll only their own line.
 enum Ctrl {
-  C_NEXT = 0,          // next chunk to claim
-  C_CNT = 1,           // C_CNT + phase: chunks of that phase completed (monotonic over units)
-  C_ROUTE = 8,         // number of units whose routing decision is published
-  C_WORDS = 16
+  C_CNT = 0,                    // C_CNT + 32*phase: chunks of that phase completed (all units)
+  C_WORDS = 32 * P_COUNT,       // every counter on its own 128-byte line
+  F_WORDS = 32                  // per-CTA flag line: word p = units whose phase p is complete
 };
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
@@ -66,15 +70,16 @@ struct Geo {
   unsigned o_ring, o_full, o_empty, o_meta, o_xr, o_xg, o_sxg, o_xs, o_sxs, o_xd, o_sxd, o_red,
       o_rows, o_misc;
   unsigned smem_bytes;
+  unsigned o_box;              // reduction slots: kBoxes x box_floats (partials + prefetched base)
+  int box_floats;
+  int red_part;                // floats of per-warp partials at the start of a slot (then bases)
 };
 
 struct Scratch {
   unsigned* ctrl;        // C_WORDS
+  unsigned* flags;       // [gridDim][F_WORDS]
   int* err;              // sticky per-device error word
   double* logits;        // [2][nr]
-  int* sidx;             // [2][K]
-  float* sw;             // [2][K]
-  float* ssig;           // [2]
   float* hs;             // [2][I]
   float* hk;             // [2][K][I]
   float* normsq;         // [n_units]

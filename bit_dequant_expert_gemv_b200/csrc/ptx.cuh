@@ -74,7 +74,34 @@ __device__ __forceinline__ int ld_volatile_int(const int* p) {
   return *reinterpret_cast<const volatile int*>(p);
 }
 
-// Barrier among the consumer warps only (id 1); the producer warp never joins it.
+// Shared-memory counter bumped with release semantics at CTA scope / read with acquire.
+__device__ __forceinline__ void red_release_cta_smem(unsigned* p, unsigned v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
+               : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+// Barrier among the consumer warps only (id 1); the producer and signal warps never join it.
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
 }

@@ -116,6 +116,35 @@ def consumer_reads(G, p, n):
                 yield "sb", b_base + b_slice + vr * b_row, 4, vr, s
 
 
+def clamped_reads(G, p):
+    """Every thread reads a clamped, in-stage address even for rows or slices it then zeroes."""
+    bits = G["bits"]
+    sbytes = 16 if bits == 4 else 8
+    K = G["K"]
+    if p in (1, 3):
+        sp, P, sl, W, vmax = G["sp_h"], G["p_h"], G["sl_h"], G["w_gu"], 2 * G["rcg"] - 1
+    elif p == 2:
+        sp, P, sl, W, vmax = G["sp_i"], G["p_i"], G["sl_i"], 4, G["rsd"] - 1
+    else:
+        sp, P, sl, W, vmax = G["sp_d"], G["p_d"], G["sl_d"], 4, G["rrd"] - 1
+    for t in range(256):
+        pp, s = divmod(t, sp)
+        sc = min(s, sl - 1)
+        for w in range(W):
+            vc = min(pp + w * P, vmax)
+            if p in (1, 3):
+                a = sc * sbytes + vc * G["rc_h"]
+                b = 2 * G["rcg"] * G["rc_h"] + (sc >> 1) * 4 + vc * G["rs_h"]
+            elif p == 2:
+                a = sc * sbytes + vc * G["rc_i"]
+                b = G["rsd"] * G["rc_i"] + (sc >> 1) * 4 + vc * G["rs_i"]
+            else:
+                kk, si = divmod(sc, G["sl_i"])
+                a = kk * G["rrd"] * G["rc_i"] + si * sbytes + vc * G["rc_i"]
+                b = K * G["rrd"] * G["rc_i"] + kk * G["rrd"] * G["rs_i"] + (si >> 1) * 4 + vc * G["rs_i"]
+            yield a, sbytes, b
+
+
 def reduce_red_extent(G, p):
     sp = {1: G["sp_h"], 3: G["sp_h"], 2: G["sp_i"], 4: G["sp_d"]}[p]
     W = G["w_gu"] if p in (1, 3) else 4
@@ -139,8 +168,8 @@ def test_geometry_in_bounds(shape, flags):
     # carve-up: ring | x areas | barriers | meta, non-overlapping and in order
     areas = [("ring", 0, ns * sb), ("xr", G["o_xr"], 4 * H), ("xg", G["o_xg"], 4 * H),
              ("sxg", G["o_sxg"], 4 * (H // 32)), ("xs", G["o_xs"], 4 * I), ("sxs", G["o_sxs"], 4 * (I // 32)),
-             ("xd", G["o_xd"], 4 * K * I), ("sxd", G["o_sxd"], 4 * K * (I // 32)), ("red", G["o_red"], 4 * 256 * KMAXW),
-             ("misc", G["o_misc"], 512), ("full", G["o_full"], 8 * ns), ("empty", G["o_empty"], 8 * ns),
+             ("xd", G["o_xd"], 4 * K * I), ("sxd", G["o_sxd"], 4 * K * (I // 32)), ("red", G["o_red"], 16),
+             ("box", G["o_box"], 4 * 4 * G["box_floats"]), ("misc", G["o_misc"], 512), ("full", G["o_full"], 8 * ns), ("empty", G["o_empty"], 8 * ns),
              ("meta", G["o_meta"], 4 * ns)]
     for (n1, a1, l1), (n2, a2, l2) in zip(areas, areas[1:]):
         assert a1 + l1 <= a2, (n1, n2)
@@ -163,7 +192,7 @@ def test_geometry_in_bounds(shape, flags):
         for (a, b), (c2, d) in zip(covered, covered[1:]):
             assert b <= c2, "copies overlap in the stage"
         if p == 0:
-            assert n <= 32 and n * 4 * H <= sb
+            assert n <= 32 and n * 4 * H <= sb and 2 * 8 * n <= G["red_part"]
             continue
         jn = G[f"n{p}"]
         if p == 3:
@@ -173,8 +202,15 @@ def test_geometry_in_bounds(shape, flags):
             continue
         for kind, off, nbytes, vr, s in consumer_reads(G, p, n):
             assert any(a <= off and off + nbytes <= b for a, b in covered), (p, kind, off, nbytes, vr, s, covered)
-        assert reduce_red_extent(G, p) <= 256 * KMAXW
-        # epilogue indices
+        assert reduce_red_extent(G, p) <= G["red_part"]
+        for a, nb, b in clamped_reads(G, p):
+            assert 0 <= a and a + nb <= sb and 0 <= b and b + 4 <= sb, (p, a, b, sb)
+        # reduction slot: partials of every segment, then one base per output row
+        nseg = lambda sp: 8 if sp >= 32 else 256 // sp
+        spp = {1: G["sp_h"], 3: G["sp_h"], 2: G["sp_i"], 4: G["sp_d"]}.get(p)
+        if spp:
+            assert nseg(spp) * KMAXW <= G["red_part"]
+        assert G["red_part"] + n <= G["box_floats"]
         if p in (1, 3):
             assert r0 + n <= I and n <= G["rcg"] and k < K
         else:
