@@ -39,7 +39,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="full_q4",
-                    choices=["full_q4", "full_q4_natural", "full_q2", "stack_q4_uniform",
+                    choices=["full_q4", "full_q4_natural", "full_q2", "tiny", "stack_q4_uniform",
                              "stack_q4_skewed", "stack_q2"])
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (0 = workload's)")
     ap.add_argument("--experts", type=int, default=0,
@@ -53,6 +53,29 @@ def parse():
 def dist_info():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
             int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The maximum of `value` over all ranks (one all-reduce; identity on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def arm_config(wl, T: int, world: int) -> dict:
+    """The `config` object of the JSON line; both arms report the same one."""
+    stack = wl.layers > 1
+    return {"workload": wl.name, "hidden": wl.H, "experts": wl.E, "top_k": wl.K,
+            "shared_experts": 1, "inter": wl.I, "bits": wl.bits, "group": 64,
+            "layers": wl.layers, "tokens_per_step": T, "routing": wl.routing,
+            "launches_per_step": 1,
+            "l2": ("inputs larger than L2: 16 round-robin copies of router/shared expert, "
+                   "512 routed experts (3.6 GB)") if not stack else
+                  "inputs larger than L2: every layer's tensors once per token",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def peaks():
@@ -181,28 +204,38 @@ def cpu_baseline(wl, seconds: float):
 
 
 def run_reference(args):
+    """The oracle arm: the plain C oracle (binary64, one thread) on this host's cores, timed on
+    a bounded sample of the same workload each step. Under torchrun only rank 0 runs it."""
     rank, _, world = dist_info()
     if rank != 0:
         return
     import synth
-    wl = synth.WORKLOADS["full_q4" if args.workload.startswith("stack") else args.workload]
-    per_step = min(args.cpu_seconds, 60.0)
-    vals = []
+    wl0 = synth.WORKLOADS[args.workload]
+    layer_wl = wl0
+    if wl0.layers > 1:  # a stack: one layer of the same shape, time scaled by the layer count
+        layer_wl = synth.WORKLOADS["full_q2" if wl0.bits == 2 else "full_q4"]
+    per_step = min(args.cpu_seconds, 60.0) / max(1, args.steps)
     for _ in range(max(1, args.warmup)):
-        cpu_baseline(wl, 1.0)
+        cpu_baseline(layer_wl, 0.5)
+    vals, samples, secs = [], [], []
     for _ in range(args.steps):
-        vals.append(cpu_baseline(wl, per_step / max(1, args.steps))["value"])
-        if len(vals) * per_step / max(1, args.steps) > 120:
+        r = cpu_baseline(layer_wl, per_step)
+        vals.append(r["value"] / wl0.layers)
+        samples.append(r["sample"])
+        secs.append(r["seconds"])
+        if len(vals) * per_step > 120:
             break
     v = statistics.median(vals)
+    sample = (f"{len(vals)} steps, each {samples[0]}"
+              + (f"; tokens/s divided by the stack's {wl0.layers} layers" if wl0.layers > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": len(vals), "warmup": args.warmup,
-            "ms_per_step": 1000.0 / v, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1000.0 * statistics.median(secs), "higher_is_better": True,
+            "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "hidden": wl.H, "experts": wl.E, "top_k": wl.K,
-                       "inter": wl.I, "bits": wl.bits, "tokens_per_step": 1},
+            "config": arm_config(wl0, args.tokens or wl0.tokens, world),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "one token per step through the oracle layer (single thread)"},
+                             "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -283,6 +316,7 @@ def run_ours(args):
     with ClockSampler(local_rank) as clk:
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed")
         start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
@@ -290,14 +324,12 @@ def run_ours(args):
             ev[i][1].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
     launches = fmoe.launch_count() - l0
     if fmoe.sync_status() != 0:
         raise RuntimeError("device status after timing: " + fmoe.last_error())
     total_ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_per_step = total_ms / args.steps
 
@@ -319,10 +351,7 @@ def run_ours(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev, world)
         h2d = xh.numel() * 4 + rh.numel() * 4 + (0 if bh is None else bh.numel() * 4)
         d2h = oh.numel() * 4
         e2e = {"value": world * T / (e2e_ms / 1000.0), "unit": "tokens/s",
@@ -344,14 +373,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp32", "data": "synthetic",
-            "config": {"workload": wl.name, "hidden": wl.H, "experts": wl.E, "top_k": wl.K,
-                       "shared_experts": 1, "inter": wl.I, "bits": wl.bits, "group": 64,
-                       "layers": wl.layers, "tokens_per_step": T, "routing": wl.routing,
-                       "launches_per_step": 1,
-                       "l2": ("inputs larger than L2: 16 round-robin copies of router/shared "
-                              "expert, 512 routed experts (3.6 GB)") if not stack else
-                             "inputs larger than L2: every layer's tensors once per token",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": arm_config(wl, T, world),
             "us_per_layer": ms_per_step * 1000.0 / layers_per_step,
             "gbs_algorithmic": bytes_per_layer * layers_per_step / (ms_per_step / 1000.0) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",

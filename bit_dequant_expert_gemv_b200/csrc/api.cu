@@ -62,6 +62,7 @@ struct DevState {
 std::mutex g_mu;
 DevState g_dev[64];
 
+
 int dev_state(DevState** out) {
   int dev = 0;
   CK(cudaGetDevice(&dev));
@@ -88,16 +89,28 @@ int dev_state(DevState** out) {
   return FMOE_OK;
 }
 
-int pad_slices(int s) {
-  if (s <= 32) {
-    int p = 1;
-    while (p < s) p <<= 1;
-    return p;
-  }
-  return (s + 31) / 32 * 32;
+unsigned align_up(unsigned v, unsigned a) { return (v + a - 1) / a * a; }
+
+// rows whose byte size times this count is a multiple of 16 (TMA bulk copy granularity)
+int rows_for_16(unsigned row_bytes) {
+  int r = 1;
+  while ((row_bytes * (unsigned)r) % 16u) r <<= 1;
+  return r;
 }
 
-unsigned align_up(unsigned v, unsigned a) { return (v + a - 1) / a * a; }
+// Lane layout of a chunk whose (virtual) rows have nsl 32-column slices and nrows rows.
+LaneMap lane_map(int nsl, int nrows) {
+  LaneMap m;
+  m.nsl = nsl;
+  m.S = 32;
+  if (nsl < 32) {
+    m.S = 1;
+    while (m.S < nsl) m.S <<= 1;
+  }
+  m.P = 32 / m.S;
+  m.nrl = (nrows + m.P - 1) / m.P;
+  return m;
+}
 
 // ---------------------------------------------------------------- validation and geometry
 int check_shape(int H, int I, int E, int K, int bits) {
@@ -112,44 +125,73 @@ int check_shape(int H, int I, int E, int K, int bits) {
   return FMOE_OK;
 }
 
+// Chunk sizes, lane layouts and the shared-memory carve-up of one launch. Each chunk kind
+// takes as many rows as fit kStageTarget bytes (at least one aligned group of rows), within
+// what one warp's lanes accumulate (kRowsPerLane rows per lane).
 int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on, bool routed_on,
              bool gate_on, int max_smem, Geo* G) {
   memset(G, 0, sizeof *G);
   G->H = H; G->I = I; G->E = E; G->K = K; G->bits = bits;
   G->route_on = route_on; G->shared_on = shared_on; G->routed_on = routed_on;
-  G->gate_on = gate_on && route_on;
+  G->gate_on = gate_on && route_on && shared_on;
   G->rc_h = (unsigned)H * bits / 8; G->rs_h = (unsigned)H / 16;
   G->rc_i = (unsigned)I * bits / 8; G->rs_i = (unsigned)I / 16;
   G->q_gu = (unsigned long long)I * (G->rc_h + G->rs_h);
-  G->q_dn = (unsigned long long)H * (G->rc_i + G->rs_i);
-  G->sl_h = H / 32; G->sp_h = pad_slices(G->sl_h); G->p_h = kConsumers / G->sp_h;
-  G->sl_i = I / 32; G->sp_i = pad_slices(G->sl_i); G->p_i = kConsumers / G->sp_i;
-  G->sl_d = K * G->sl_i; G->sp_d = pad_slices(G->sl_d); G->p_d = kConsumers / G->sp_d;
-  if (G->sp_h > kMaxSlices || G->sp_i > kMaxSlices || G->sp_d > kMaxSlices || G->p_h < 1 ||
-      G->p_i < 1 || G->p_d < 1)
-    return fail(FMOE_ERR_UNSUPPORTED, "row too wide for one CTA (H=%d I=%d K=%d)", H, I, K);
-  G->w_gu = G->p_h == 1 ? 8 : 4;
-  G->w_sd = 4;
-  G->w_rd = 4;
-  G->rcg = G->w_gu * G->p_h / 2;
-  G->rsd = 4 * G->p_i;
-  G->rrd = 4 * G->p_d;
+  const unsigned cap = (unsigned)kStageTarget;
+  // router: whole rows when a row fits, else column segments of one row
   G->nr = route_on ? E + (G->gate_on ? 1 : 0) : 0;
-  G->rr = std::max(1, std::min(32, 16384 / (4 * H)));
-  G->nb = (I + G->rcg - 1) / G->rcg;
-  G->n[P_ROUTER] = route_on ? (G->nr + G->rr - 1) / G->rr : 0;
-  G->n[P_SGU] = shared_on ? G->nb : 0;
-  G->n[P_SDN] = shared_on ? (H + G->rsd - 1) / G->rsd : 0;
-  G->n[P_RGU] = routed_on ? K * G->nb : 0;
-  G->n[P_RDN] = routed_on ? (H + G->rrd - 1) / G->rrd : 0;
+  if (4u * H <= cap) {
+    G->rseg = 1;
+    G->rcols = H;
+    G->rrows = std::max(1, std::min(64, (int)(cap / (4u * H))));
+  } else {
+    int d = (int)((4u * H + cap - 1) / cap);
+    while (H % d || (H / d) % 4) ++d;
+    G->rseg = d;
+    G->rcols = H / d;
+    G->rrows = 1;
+  }
+  G->nrb = G->nr ? (G->nr + G->rrows - 1) / G->rrows : 0;
+  // gate/up: R rows of gate and R of up per chunk
+  {
+    const int al = std::max(rows_for_16(G->rc_h), rows_for_16(G->rs_h));
+    const LaneMap m1 = lane_map(H / 32, 1);
+    int r = (int)(cap / (2u * (G->rc_h + G->rs_h)));
+    r = std::min(r, kRowsPerLane * m1.P / 2);
+    r = std::min(r, I);
+    r = std::max(al, r / al * al);
+    G->R = r;
+    G->nb = (I + r - 1) / r;
+    G->gu = lane_map(H / 32, 2 * r);
+  }
+  // down: Rd virtual rows of nseg segments per chunk
+  G->nseg = (shared_on ? 1 : 0) + (routed_on ? K : 0);
+  if (G->nseg > 0) {
+    const int al = std::max(rows_for_16(G->rc_i), rows_for_16(G->rs_i));
+    const LaneMap m1 = lane_map(G->nseg * I / 32, 1);
+    int r = (int)(cap / ((unsigned)G->nseg * (G->rc_i + G->rs_i)));
+    r = std::min(r, kRowsPerLane * m1.P);
+    r = std::min(r, H);
+    r = std::max(al, r / al * al);
+    G->Rd = r;
+    G->dn = lane_map(G->nseg * I / 32, r);
+  }
+  if (G->gu.nrl > kRowsPerLane || G->dn.nrl > kRowsPerLane)
+    return fail(FMOE_ERR_UNSUPPORTED, "row layout too wide (H=%d I=%d K=%d)", H, I, K);
+  G->n[K_ROUTER] = route_on ? G->nrb * G->rseg : 0;
+  G->n[K_SGU] = shared_on ? G->nb : 0;
+  G->n[K_RGU] = routed_on ? K * G->nb : 0;
+  G->n[K_DN] = G->nseg > 0 ? (H + G->Rd - 1) / G->Rd : 0;
   G->off[0] = 0;
-  for (int p = 0; p < P_COUNT; ++p) G->off[p + 1] = G->off[p] + G->n[p];
-  if (G->off[P_COUNT] == 0) return fail(FMOE_ERR_INVALID, "nothing to compute");
+  for (int k = 0; k < K_COUNT; ++k) G->off[k + 1] = G->off[k] + G->n[k];
+  if (G->off[K_COUNT] == 0) return fail(FMOE_ERR_INVALID, "nothing to compute");
+  G->ncl[CL_ROUTER] = G->n[K_ROUTER];
+  G->ncl[CL_GU] = G->n[K_SGU] + G->n[K_RGU];
+  G->ncl[CL_DN] = G->n[K_DN];
   unsigned stage = 0;
-  if (route_on) stage = std::max(stage, (unsigned)G->rr * 4u * H);
-  if (shared_on || routed_on) stage = std::max(stage, 2u * G->rcg * (G->rc_h + G->rs_h));
-  if (shared_on) stage = std::max(stage, (unsigned)G->rsd * (G->rc_i + G->rs_i));
-  if (routed_on) stage = std::max(stage, (unsigned)K * G->rrd * (G->rc_i + G->rs_i));
+  if (route_on) stage = std::max(stage, (unsigned)G->rrows * 4u * G->rcols);
+  if (shared_on || routed_on) stage = std::max(stage, 2u * G->R * (G->rc_h + G->rs_h));
+  if (G->nseg > 0) stage = std::max(stage, (unsigned)G->Rd * G->nseg * (G->rc_i + G->rs_i));
   G->stage_bytes = align_up(stage, 128);
   // fixed areas after the ring
   unsigned o = 0;
@@ -158,39 +200,27 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
     o = align_up(o + bytes, 128);
     return at;
   };
-  G->o_xr = take(4u * H);
-  G->o_xg = take(4u * H);
-  G->o_sxg = take(4u * G->sl_h);
-  G->o_xs = take(4u * I);
-  G->o_sxs = take(4u * G->sl_i);
-  G->o_xd = take(4u * K * I);
-  G->o_sxd = take(4u * G->sl_d);
-  // reduction slot: per-warp (or per-segment) row partials, kMaxW per segment; router rows
-  // as binary64 partials of 8 warps x rr rows; then one prefetched base per output row
-  auto nseg = [](int sp) { return sp >= 32 ? kConsumerWarps : kConsumers / sp; };
-  const int part = std::max(std::max(nseg(G->sp_h), std::max(nseg(G->sp_i), nseg(G->sp_d))) * 8,
-                            2 * kConsumerWarps * G->rr);
-  G->red_part = (part + 31) / 32 * 32;
-  G->box_floats = G->red_part + (std::max(G->rsd, G->rrd) + 31) / 32 * 32;
-  G->o_red = take(16);
-  G->o_box = take(4u * kBoxes * G->box_floats);
+  G->o_xa = take(4u * (unsigned)std::max(H, G->nseg * I));  // x (raw) / down input (transformed)
+  G->o_sxa = take(4u * (unsigned)std::max(1, G->nseg * I / 32));
+  G->o_xg = take(4u * H);                                     // x transformed
+  G->o_sxg = take(4u * (H / 32));
+  G->o_red = take(4u * kConsumerWarps * 16 * kRowsPerLane);   // per-warp row sums
   G->o_misc = take(512);
   const unsigned fixed = o;
-  const unsigned avail = (unsigned)max_smem - 1024;  // slack for alignment of the base
-  if (fixed + 2 * G->stage_bytes + 2 * 16 * 2 + 64 > avail)
+  const unsigned avail = (unsigned)max_smem;
+  if (fixed + 2 * (G->stage_bytes + 16) > avail)
     return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for two stages");
-  int ns = (int)((avail - fixed - 256) / (G->stage_bytes + 20));
-  ns = std::min(ns, 16);
+  int ns = (int)((avail - fixed) / (G->stage_bytes + 16));
+  ns = std::min(ns, kMaxStages);
   G->nstage = ns;
-  // final layout: ring | x areas (shifted) | barriers | meta
+  // final layout: ring | fixed areas | barriers
   const unsigned ring = (unsigned)ns * G->stage_bytes;
   G->o_ring = 0;
-  G->o_xr += ring; G->o_xg += ring; G->o_sxg += ring; G->o_xs += ring; G->o_sxs += ring;
-  G->o_xd += ring; G->o_sxd += ring; G->o_red += ring; G->o_misc += ring; G->o_box += ring;
-  G->o_full = align_up(ring + fixed, 128);
+  G->o_xa += ring; G->o_sxa += ring; G->o_xg += ring; G->o_sxg += ring; G->o_red += ring;
+  G->o_misc += ring;
+  G->o_full = ring + fixed;
   G->o_empty = G->o_full + 8u * ns;
-  G->o_meta = G->o_empty + 8u * ns;
-  G->smem_bytes = align_up(G->o_meta + 4u * ns, 128);
+  G->smem_bytes = G->o_empty + 8u * ns;
   if (G->smem_bytes > (unsigned)max_smem)
     return fail(FMOE_ERR_UNSUPPORTED, "shared memory layout too large (%u)", G->smem_bytes);
   return FMOE_OK;
@@ -227,7 +257,7 @@ ScratchPlan plan_scratch(const Geo& G, int n_units, int max_grid) {
   s.off_flags = o; o = up256(o + 4 * (size_t)F_WORDS * max_grid);
   s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
   s.zero_bytes = o;
-  s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.nr, 1));
+  s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.rseg, 1) * std::max(G.nr, 1));
   s.off_hs = o; o = up256(o + 4 * 2 * (size_t)G.I);
   s.off_hk = o; o = up256(o + 4 * 2 * (size_t)G.K * G.I);
   s.off_hbuf = o; o = up256(o + 4 * 2 * (size_t)G.H);
@@ -260,7 +290,7 @@ void fill_layers(Prog* P, const fmoe_layer_desc* layers, int n) {
 int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, int sms,
                    cudaStream_t st) {
   CK(cudaMemsetAsync(base, 0, sp.zero_bytes, st));
-  const long long total = (long long)P->n_units * G.off[P_COUNT];
+  const long long total = (long long)P->n_units * G.off[K_COUNT];
   const int grid = (int)std::min<long long>(sms, std::max<long long>(1, total));
   cudaError_t e = fmoe_engine_launch(P, &G, grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "engine launch");
@@ -313,14 +343,12 @@ int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int 
                      flags & 8, max_smem, &G)))
     return rc;
   const int64_t v[] = {G.H, G.I, G.E, G.K, G.bits, G.route_on, G.shared_on, G.routed_on,
-                       G.gate_on, G.rc_h, G.rs_h, G.rc_i, G.rs_i, (int64_t)G.q_gu,
-                       (int64_t)G.q_dn, G.rr, G.rcg, G.rsd, G.rrd, G.nr, G.nb, G.n[0], G.n[1],
-                       G.n[2], G.n[3], G.n[4], G.off[0], G.off[1], G.off[2], G.off[3], G.off[4],
-                       G.off[5], G.sl_h, G.sp_h, G.p_h, G.sl_i, G.sp_i, G.p_i, G.sl_d, G.sp_d,
-                       G.p_d, G.w_gu, G.w_sd, G.w_rd, G.stage_bytes, G.nstage, G.o_ring,
-                       G.o_full, G.o_empty, G.o_meta, G.o_xr, G.o_xg, G.o_sxg, G.o_xs, G.o_sxs,
-                       G.o_xd, G.o_sxd, G.o_red, G.o_misc, G.smem_bytes, G.o_box,
-                       G.box_floats, G.red_part};
+                       G.gate_on, G.rc_h, G.rs_h, G.rc_i, G.rs_i, (int64_t)G.q_gu, G.nr, G.rseg,
+                       G.rcols, G.rrows, G.nrb, G.R, G.nb, G.nseg, G.Rd, G.n[0], G.n[1], G.n[2],
+                       G.n[3], G.off[0], G.off[1], G.off[2], G.off[3], G.off[4], G.ncl[0],
+                       G.ncl[1], G.ncl[2], G.gu.nsl, G.gu.S, G.gu.P, G.gu.nrl, G.dn.nsl, G.dn.S,
+                       G.dn.P, G.dn.nrl, G.stage_bytes, G.nstage, G.o_ring, G.o_full, G.o_empty,
+                       G.o_xa, G.o_sxa, G.o_xg, G.o_sxg, G.o_red, G.o_misc, G.smem_bytes};
   const int n = (int)(sizeof v / sizeof v[0]);
   for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
   return n < n_out ? n : n_out;
@@ -447,7 +475,7 @@ int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float*
   Geo G;
   if ((rc = prep_layers(layers, n_layers, d, &G))) return rc;
   if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
-  if ((long long)n_tokens * G.off[P_COUNT] > 0x7ffffff0ll) return fail(FMOE_ERR_UNSUPPORTED, "too many tokens");
+  if ((long long)n_tokens * G.off[K_COUNT] > 0x7ffffff0ll) return fail(FMOE_ERR_UNSUPPORTED, "too many tokens");
   if (!x || !out) return fail(FMOE_ERR_INVALID, "x and out are required");
   if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
     return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
@@ -520,7 +548,7 @@ static int stack_prog(const fmoe_layer_desc* layers, int n_layers, const float* 
   int rc = prep_layers(layers, n_layers, d, G);
   if (rc) return rc;
   if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
-  if ((long long)n_tokens * n_layers * G->off[P_COUNT] > 0x7ffffff0ll)
+  if ((long long)n_tokens * n_layers * G->off[K_COUNT] > 0x7ffffff0ll)
     return fail(FMOE_ERR_UNSUPPORTED, "too many tokens x layers for one launch");
   if (!h_in || !h_out) return fail(FMOE_ERR_INVALID, "h_in and h_out are required");
   if (!aligned16(h_in) || !aligned16(h_out) || !aligned16(h_trace))

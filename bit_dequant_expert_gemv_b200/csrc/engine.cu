@@ -15,21 +15,24 @@
 //     "Qu'est-ce que Flash-MoE ?" (a2a-mcp.org, fr), §2 "Noyaux de Déquantification Optimisés
 //      pour FMA").
 //
-// How: one CTA per SM with three roles.
-//   producer warp   streams the weight rows of the CTA's chunks into a ring of shared-memory
-//                   stages with 1-D TMA bulk copies completing on mbarriers;
-//   8 consumer warps own fixed 32-column slices, keep the matching (pre-transformed) x values
-//                   in registers, unpack codes with one byte-permute per byte into a binary32
-//                   "32768 + byte" pattern and finish the exact code values with packed f32x2
-//                   arithmetic; row partials are reduced with a transposing warp butterfly and
-//                   across warps in shared memory, then the epilogue (SwiGLU or combine) runs;
-//   signal warp     moves each chunk's epilogue results from a shared-memory outbox to global
-//                   memory, publishes completions to the other CTAs (one gpu-scope fence and
-//                   one reduction per run of same-phase chunks) and, in the CTA that completes
-//                   the router, selects the top-K experts -- so the consumers never wait on a
-//                   global store, fence or atomic.
-// Every spin-wait is bounded by a global-timer budget; on expiry the kernel records an error
-// word, waits for its own copies in flight and returns.
+// How: one CTA per SM, every CTA working through a static share of every unit's chunks.
+//   producer warp   streams each chunk's weight rows into a ring of shared-memory stages with
+//                   1-D TMA bulk copies that complete on the stage's mbarrier;
+//   stager warp     per unit: brings x into shared memory (TMA) and prepares its two forms
+//                   (raw for the router, pair-transformed + slice sums for the codes), selects
+//                   the top-K experts once the router is complete, and prepares the down
+//                   input [sigma*h_s | w_k*h_k] once every gate/up chunk is complete;
+//   consumer warps  each owns whole chunks (local chunk i -> warp i mod kConsumerWarps):
+//                   unpacks codes with one byte-permute per byte into a binary32
+//                   "32768 + byte" pattern, finishes the exact code values with packed f32x2
+//                   arithmetic, reduces its row sums inside the warp and runs the chunk's
+//                   epilogue (logit store, SwiGLU, or residual + combine) itself -- no
+//                   block-wide barrier and no cross-warp reduction on the hot path.
+// Completion is published per run of same-class chunks of a CTA: the warp finishing a run's
+// last chunk makes one gpu-scope fence and one atomic, and the CTA completing a class for a
+// unit writes a flag into every CTA's own flag line. Every spin-wait is bounded by a
+// global-timer budget; on expiry the kernel records an error word, waits for its own copies
+// in flight and returns.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -38,15 +41,8 @@
 
 namespace fmoe {
 
-constexpr int kMaxW = 8;
-// Warp roles: warp 0 producer, warp 1 signal, warps 2..9 consumers. The control warps get the
-// lowest warp ids so that, sharing sub-partitions with busy consumer warps, they are not
-// starved of issue slots.
-constexpr int kCtrlThreads = 64;
-__device__ __forceinline__ int ctid() { return (int)threadIdx.x - kCtrlThreads; }
-
-__device__ __forceinline__ int cnt_word(int phase) { return C_CNT + 32 * phase; }
-// this CTA's flag word `w` (units whose phase w is complete)
+__device__ __forceinline__ int cnt_word(int cls) { return C_CNT + 32 * cls; }
+// this CTA's flag word `w` (units whose class w is complete)
 __device__ __forceinline__ const unsigned* my_flag(const Prog& P, int w) {
   return P.s.flags + blockIdx.x * F_WORDS + w;
 }
@@ -99,75 +95,93 @@ __device__ __forceinline__ UnitView unit_view(const Prog& P, const Geo& G, int u
   return v;
 }
 
-struct ChunkView {
-  int u, c, phase, j, r0, n, k;
+struct Chunk {
+  int u, c, kind, j, r0, n, k, seg;
 };
 
-// The chunks of this CTA in order: g = blockIdx + it * gridDim, decoded incrementally.
-struct ChunkIter {
-  unsigned it, total;
-  int u, c, ntot, step;
-  __device__ __forceinline__ ChunkIter(const Prog& P, const Geo& G) {
-    ntot = G.off[P_COUNT];
-    total = (unsigned)P.n_units * (unsigned)ntot;
-    step = (int)gridDim.x;
-    it = 0;
-    u = (int)(blockIdx.x / (unsigned)ntot);
-    c = (int)(blockIdx.x - (unsigned)u * (unsigned)ntot);
-  }
-  __device__ __forceinline__ bool valid() const {
-    return (unsigned)u * (unsigned)ntot + (unsigned)c < total;
-  }
-  __device__ __forceinline__ void next() {
-    ++it;
-    c += step;
-    while (c >= ntot) {
-      c -= ntot;
-      ++u;
+__device__ __forceinline__ Chunk chunk_at(const Geo& G, unsigned long long g) {
+  const unsigned ntot = (unsigned)G.off[K_COUNT];
+  Chunk v;
+  v.u = (int)(g / ntot);
+  v.c = (int)(g - (unsigned long long)v.u * ntot);
+  int kd = 0;
+  while (v.c >= G.off[kd + 1]) ++kd;
+  v.kind = kd;
+  v.j = v.c - G.off[kd];
+  v.k = 0;
+  v.seg = 0;
+  switch (kd) {
+    case K_ROUTER: {
+      const int rb = v.j / G.rseg;
+      v.seg = v.j - rb * G.rseg;
+      v.r0 = rb * G.rrows;
+      v.n = min(G.rrows, G.nr - v.r0);
+      break;
     }
+    case K_SGU:
+      v.r0 = v.j * G.R;
+      v.n = min(G.R, G.I - v.r0);
+      break;
+    case K_RGU:
+      v.k = v.j / G.nb;
+      v.r0 = (v.j - v.k * G.nb) * G.R;
+      v.n = min(G.R, G.I - v.r0);
+      break;
+    default:
+      v.r0 = v.j * G.Rd;
+      v.n = min(G.Rd, G.H - v.r0);
+      break;
   }
-  __device__ __forceinline__ ChunkView view(const Geo& G) const {
-    ChunkView v;
-    v.u = u;
-    v.c = c;
-    int p = 0;
-    while (c >= G.off[p + 1]) ++p;
-    v.phase = p;
-    v.j = c - G.off[p];
-    v.k = 0;
-    switch (p) {
-      case P_ROUTER: v.r0 = v.j * G.rr; v.n = min(G.rr, G.nr - v.r0); break;
-      case P_SGU: v.r0 = v.j * G.rcg; v.n = min(G.rcg, G.I - v.r0); break;
-      case P_SDN: v.r0 = v.j * G.rsd; v.n = min(G.rsd, G.H - v.r0); break;
-      case P_RGU: {
-        v.k = v.j / G.nb;
-        const int jj = v.j - v.k * G.nb;
-        v.r0 = jj * G.rcg;
-        v.n = min(G.rcg, G.I - v.r0);
-        break;
-      }
-      default: v.r0 = v.j * G.rrd; v.n = min(G.rrd, G.H - v.r0); break;
-    }
-    return v;
-  }
-};
+  return v;
+}
 
-// the phase whose completion means "the unit is complete"
-__device__ __forceinline__ int final_phase(const Geo& G) {
-  return G.routed_on ? P_RDN : (G.shared_on ? P_SDN : P_ROUTER);
+__device__ __forceinline__ int class_of(int kind) {
+  return kind == K_ROUTER ? CL_ROUTER : (kind == K_DN ? CL_DN : CL_GU);
+}
+
+// the class whose completion means "the unit is complete"
+__device__ __forceinline__ int final_class(const Geo& G) {
+  return G.nseg > 0 ? CL_DN : CL_ROUTER;
+}
+
+__device__ __forceinline__ int class_lo(const Geo& G, int cls) {
+  return cls == CL_ROUTER ? G.off[K_ROUTER] : (cls == CL_GU ? G.off[K_SGU] : G.off[K_DN]);
+}
+__device__ __forceinline__ int class_hi(const Geo& G, int cls) {
+  return cls == CL_ROUTER ? G.off[K_SGU] : (cls == CL_GU ? G.off[K_DN] : G.off[K_COUNT]);
+}
+
+// number of x in [lo, hi) with x mod m == r (r < m)
+__device__ __forceinline__ unsigned count_cong(unsigned long long lo, unsigned long long hi,
+                                               unsigned r, unsigned m) {
+  const unsigned long long a = lo > r ? (lo - r + m - 1) / m : 0ull;
+  const unsigned long long b = hi > r ? (hi - r + m - 1) / m : 0ull;
+  return (unsigned)(b - a);
+}
+
+// chunks of class `cls` of unit u that belong to this CTA
+__device__ __forceinline__ unsigned run_len(const Geo& G, int u, int cls) {
+  const unsigned long long base = (unsigned long long)u * (unsigned)G.off[K_COUNT];
+  return count_cong(base + class_lo(G, cls), base + class_hi(G, cls), blockIdx.x, gridDim.x);
+}
+
+__device__ __forceinline__ unsigned local_chunks(const Prog& P, const Geo& G) {
+  const unsigned long long total = (unsigned long long)P.n_units * (unsigned)G.off[K_COUNT];
+  return count_cong(0ull, total, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------------------------------------------------
 // bounded waits
 // ------------------------------------------------------------------------------------------
 struct Smem {  // small shared state (in the misc area)
+  uint64_t xbar;               // the stager's TMA barrier
   volatile int abort;
-  volatile int prod_done;
-  volatile unsigned issued;
-  unsigned done_count;         // consumer warps x chunks completed (CTA-scope release counter)
-  volatile unsigned sig_done;  // chunks whose outbox the signal warp has emptied
-  volatile int cons_done;
-  int rt_e[2][kMaxK];    // routing of units u (index u & 1): experts and weights, by the producer
+  unsigned x_ready;            // units whose x is staged          (release/acquire, CTA)
+  unsigned rt_ready;           // units whose routing is in rt_*   (release/acquire, CTA)
+  unsigned xd_ready;           // units whose down input is staged (release/acquire, CTA)
+  unsigned run_cnt[CL_COUNT];  // chunks of the current run of each class finished here
+  volatile unsigned issued;    // chunks the producer has issued
+  int rt_e[2][kMaxK];          // routing of unit u (index u & 1): experts and weights
   float rt_w[2][kMaxK];
 };
 
@@ -176,7 +190,8 @@ __device__ __forceinline__ void raise_error(const Prog& P, Smem* sm, int code) {
   sm->abort = 1;
 }
 
-// Spin until ctrl[word] - target >= 0 (wrap-safe), the budget runs out or an abort is seen.
+// Spin until *a - target >= 0 (wrap-safe) on a gpu-scope flag, the budget runs out, the CTA
+// aborts or another CTA has recorded an error.
 __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a, unsigned target,
                                       int code) {
   if ((int)(ld_acquire(a) - target) >= 0) return true;
@@ -194,7 +209,23 @@ __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a
         return false;
       }
     }
-    __nanosleep(100);
+    __nanosleep(64);
+  }
+}
+
+// Same on a CTA-local counter in shared memory.
+__device__ __noinline__ bool spin_geq_smem(const Prog& P, Smem* sm, const unsigned* a,
+                                           unsigned target, int code) {
+  if ((int)(ld_acquire_cta_smem(a) - target) >= 0) return true;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+  for (unsigned it = 0;; ++it) {
+    if ((int)(ld_acquire_cta_smem(a) - target) >= 0) return true;
+    if (sm->abort) return false;
+    if ((it & 63) == 63 && global_ns() > deadline) {
+      raise_error(P, sm, code);
+      return false;
+    }
+    __nanosleep(32);
   }
 }
 
@@ -205,133 +236,179 @@ __device__ __forceinline__ bool wait_mbar(const Prog& P, Smem* sm, uint64_t* bar
   for (unsigned it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (sm->abort) return false;
-    if ((it & 63) == 63) {
-      if (ld_volatile_int(P.s.err) != 0) {
-        sm->abort = 1;
-        return false;
-      }
-      if (global_ns() > deadline) {
-        raise_error(P, sm, code);
-        return false;
-      }
+    if ((it & 63) == 63 && global_ns() > deadline) {
+      raise_error(P, sm, code);
+      return false;
     }
   }
 }
 
-// Consumer-wide wait: thread 0 spins, all consumers get the same verdict at the barrier.
-__device__ __forceinline__ bool consumer_wait(const Prog& P, Smem* sm, int word, unsigned target,
-                                              int code) {
-  if (ctid() == 0) spin_geq(P, sm, my_flag(P, word), target, code);
-  return !consumer_any(sm->abort != 0);
+// Whole-warp wrappers: lane 0 waits, every lane gets the verdict, and what was published
+// before the flag is visible to every lane afterwards.
+__device__ __forceinline__ bool warp_wait_flag(const Prog& P, Smem* sm, int cls, unsigned target,
+                                               int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = spin_geq(P, sm, my_flag(P, cls), target, code);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_smem(const Prog& P, Smem* sm, const unsigned* a,
+                                               unsigned target, int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = spin_geq_smem(P, sm, a, target, code);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t* bar,
+                                               unsigned parity, int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_mbar(P, sm, bar, parity, code);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
 }
 
 // ------------------------------------------------------------------------------------------
-// producer: stream the rows of this CTA's chunks into the ring
+// completion of a chunk: counted per run of same-class chunks, published per run
 // ------------------------------------------------------------------------------------------
-__device__ __forceinline__ void stage_rows(uint8_t* dst, const uint8_t* src, unsigned bytes,
-                                           uint64_t* bar) {
+// Called by the whole warp after every global store of the chunk was issued. The warp whose
+// chunk completes its CTA's run of (unit, class) orders the run's stores of every warp of the
+// CTA (CTA-scope acquire of the run counter, then a gpu-scope fence) before its atomic on the
+// class counter; the warp whose atomic completes the class for the unit writes the flag of
+// every CTA (release stores).
+__device__ __forceinline__ void finish_chunk(const Prog& P, const Geo& G, Smem* sm, int cls,
+                                             int u) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  int bcast = 0;
+  if (lane == 0) {
+    const unsigned old = atom_add_acq_rel_cta_smem(&sm->run_cnt[cls], 1u);
+    const unsigned nrun = run_len(G, u, cls);
+    if (old + 1u == nrun) {
+      atom_exch_cta_smem(&sm->run_cnt[cls], 0u);
+      fence_acq_rel_gpu();
+      const unsigned og = atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cls), nrun);
+      bcast = og + nrun == (unsigned)(u + 1) * (unsigned)G.ncl[cls];
+    }
+  }
+  bcast = __shfl_sync(0xffffffffu, bcast, 0);
+  if (bcast && !(cls == CL_ROUTER && (P.debug & 1))) {
+    __syncwarp();
+    for (int c = lane; c < (int)gridDim.x; c += 32)
+      st_release(P.s.flags + c * F_WORDS + cls, (unsigned)(u + 1));
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// producer: stream the rows of this CTA's chunks into the ring (lane 0 of warp 0)
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void copy_rows(uint8_t* dst, const uint8_t* src, unsigned bytes,
+                                          uint64_t* bar) {
   if (bytes) tma_load_1d(dst, src, bytes, bar);
 }
 
-__device__ void topk_warp(const Prog& P, const Geo& G, int u, int slot, const float* bias,
-                          int* idx_out, float* w_out, Smem* sm);
-
-// The whole producer warp runs this loop; lane 0 issues the copies, and all 32 lanes select
-// the top-K experts of a unit when its first routed chunk comes up (every CTA computes the
-// same selection from the same logits, so no second broadcast is needed).
 __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
-  const int lane = threadIdx.x & 31;
-  const int NS = G.nstage;
-  int route_unit = -1;
+  const unsigned NS = (unsigned)G.nstage;
+  const unsigned n_local = local_chunks(P, G);
+  int rt_u = -1;
   int eidx[kMaxK];
-  for (ChunkIter ci(P, G); ci.valid(); ci.next()) {
-    const unsigned it = ci.it;
-    const int slot = (int)(it % NS);
-    const unsigned ph = (it / NS) & 1u;
-    int ok = 1;
-    if (lane == 0) ok = wait_mbar(P, sm, &empty[slot], ph ^ 1u, DE_TIMEOUT_EMPTY);
-    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-    const ChunkView cv = ci.view(G);
-    const UnitView uv = unit_view(P, G, cv.u);
-    const LayerW& L = *uv.L;
-    if ((cv.phase == P_RGU || cv.phase == P_RDN) && route_unit != cv.u) {
-      if (lane == 0) ok = spin_geq(P, sm, my_flag(P, P_ROUTER), (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      // the CTA owning the unit's first routed chunk writes the caller's routing outputs
-      const unsigned first = (unsigned)cv.u * (unsigned)ci.ntot + (unsigned)G.off[P_RGU];
-      const bool outs = first % gridDim.x == blockIdx.x;
-      topk_warp(P, G, cv.u, uv.slot, uv.bias, outs ? uv.idx_out : nullptr,
-                outs ? uv.w_out : nullptr, sm);
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) eidx[k] = 0;
+  unsigned i = 0;
+  for (; i < n_local; ++i) {
+    const int slot = (int)(i % NS);
+    if (!wait_mbar(P, sm, &empty[slot], ((i / NS) & 1u) ^ 1u, DE_TIMEOUT_EMPTY)) break;
+    const Chunk cv =
+        chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
+    const bool routed = cv.kind == K_RGU || (cv.kind == K_DN && G.routed_on);
+    if (routed && cv.u != rt_u) {
+      if (!spin_geq_smem(P, sm, &sm->rt_ready, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE)) break;
       for (int k = 0; k < G.K; ++k) eidx[k] = min(max(sm->rt_e[cv.u & 1][k], 0), G.E - 1);
-      route_unit = cv.u;
+      rt_u = cv.u;
     }
-    if (lane == 0) {
-      uint8_t* dst = smem + G.o_ring + (size_t)slot * G.stage_bytes;
-      switch (cv.phase) {
-        case P_ROUTER: {
-          const unsigned rowb = 4u * G.H;
+    const LayerW& L = P.layers[cv.u % P.n_layers];
+    uint8_t* dst = smem + G.o_ring + (size_t)slot * G.stage_bytes;
+    switch (cv.kind) {
+      case K_ROUTER: {
+        if (G.rseg == 1) {  // whole rows r0 .. r0+n-1; row E is the shared-gate vector
+          const unsigned rowb = 4u * (unsigned)G.H;
           const int a = cv.r0, b = min(cv.r0 + cv.n, G.E);
-          const unsigned bytes =
-              (b > a ? (unsigned)(b - a) * rowb : 0u) + (cv.r0 + cv.n > G.E ? rowb : 0u);
+          const bool gate_row = cv.r0 + cv.n > G.E;
+          const unsigned bytes = (b > a ? (unsigned)(b - a) * rowb : 0u) + (gate_row ? rowb : 0u);
           mbar_arrive_expect_tx(&full[slot], bytes);
           if (b > a)
-            stage_rows(dst, reinterpret_cast<const uint8_t*>(L.router + (size_t)a * G.H),
-                       (unsigned)(b - a) * rowb, &full[slot]);
-          if (cv.r0 + cv.n > G.E)
-            stage_rows(dst + (size_t)(G.E - cv.r0) * rowb,
-                       reinterpret_cast<const uint8_t*>(L.gate), rowb, &full[slot]);
-          break;
+            copy_rows(dst, reinterpret_cast<const uint8_t*>(L.router + (size_t)a * G.H),
+                      (unsigned)(b - a) * rowb, &full[slot]);
+          if (gate_row)
+            copy_rows(dst + (size_t)(G.E - cv.r0) * rowb, reinterpret_cast<const uint8_t*>(L.gate),
+                      rowb, &full[slot]);
+        } else {  // one column segment of row r0
+          const float* row = cv.r0 < G.E ? L.router + (size_t)cv.r0 * G.H : L.gate;
+          const unsigned bytes = 4u * (unsigned)G.rcols;
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          copy_rows(dst, reinterpret_cast<const uint8_t*>(row + (size_t)cv.seg * G.rcols), bytes,
+                    &full[slot]);
         }
-        case P_SGU:
-        case P_RGU: {
-          const uint8_t* base =
-              cv.phase == P_SGU ? L.shared : L.experts + (size_t)eidx[cv.k] * L.expert_stride;
-          const unsigned cb = (unsigned)cv.n * G.rc_h, sbb = (unsigned)cv.n * G.rs_h;
-          mbar_arrive_expect_tx(&full[slot], 2u * (cb + sbb));
-          const size_t sbo = (size_t)G.I * G.rc_h;
-          stage_rows(dst, base + (size_t)cv.r0 * G.rc_h, cb, &full[slot]);
-          stage_rows(dst + (size_t)G.rcg * G.rc_h, base + G.q_gu + (size_t)cv.r0 * G.rc_h, cb,
-                     &full[slot]);
-          uint8_t* dsb = dst + (size_t)2 * G.rcg * G.rc_h;
-          stage_rows(dsb, base + sbo + (size_t)cv.r0 * G.rs_h, sbb, &full[slot]);
-          stage_rows(dsb + (size_t)G.rcg * G.rs_h,
-                     base + G.q_gu + sbo + (size_t)cv.r0 * G.rs_h, sbb, &full[slot]);
-          break;
+        break;
+      }
+      case K_SGU:
+      case K_RGU: {  // stage: gate codes | up codes | gate sb | up sb, R rows each
+        const uint8_t* base =
+            cv.kind == K_SGU ? L.shared : L.experts + (size_t)eidx[cv.k] * L.expert_stride;
+        const unsigned cb = (unsigned)cv.n * G.rc_h, sbb = (unsigned)cv.n * G.rs_h;
+        mbar_arrive_expect_tx(&full[slot], 2u * (cb + sbb));
+        const size_t sbo = (size_t)G.I * G.rc_h;
+        copy_rows(dst, base + (size_t)cv.r0 * G.rc_h, cb, &full[slot]);
+        copy_rows(dst + (size_t)G.R * G.rc_h, base + G.q_gu + (size_t)cv.r0 * G.rc_h, cb,
+                  &full[slot]);
+        uint8_t* dsb = dst + (size_t)2 * G.R * G.rc_h;
+        copy_rows(dsb, base + sbo + (size_t)cv.r0 * G.rs_h, sbb, &full[slot]);
+        copy_rows(dsb + (size_t)G.R * G.rs_h, base + G.q_gu + sbo + (size_t)cv.r0 * G.rs_h, sbb,
+                  &full[slot]);
+        break;
+      }
+      default: {  // K_DN: per segment (shared first, then routed k) Rd rows of codes | sb
+        const unsigned cb = (unsigned)cv.n * G.rc_i, sbb = (unsigned)cv.n * G.rs_i;
+        mbar_arrive_expect_tx(&full[slot], (unsigned)G.nseg * (cb + sbb));
+        uint8_t* dsb = dst + (size_t)G.nseg * G.Rd * G.rc_i;
+        for (int s = 0; s < G.nseg; ++s) {
+          const uint8_t* eb = (G.shared_on && s == 0)
+                                  ? L.shared
+                                  : L.experts + (size_t)eidx[s - G.shared_on] * L.expert_stride;
+          const uint8_t* dn = eb + 2 * G.q_gu;
+          copy_rows(dst + (size_t)s * G.Rd * G.rc_i, dn + (size_t)cv.r0 * G.rc_i, cb, &full[slot]);
+          copy_rows(dsb + (size_t)s * G.Rd * G.rs_i,
+                    dn + (size_t)G.H * G.rc_i + (size_t)cv.r0 * G.rs_i, sbb, &full[slot]);
         }
-        case P_SDN: {
-          const uint8_t* base = L.shared + 2 * G.q_gu;
-          const unsigned cb = (unsigned)cv.n * G.rc_i, sbb = (unsigned)cv.n * G.rs_i;
-          mbar_arrive_expect_tx(&full[slot], cb + sbb);
-          stage_rows(dst, base + (size_t)cv.r0 * G.rc_i, cb, &full[slot]);
-          stage_rows(dst + (size_t)G.rsd * G.rc_i,
-                     base + (size_t)G.H * G.rc_i + (size_t)cv.r0 * G.rs_i, sbb, &full[slot]);
-          break;
-        }
-        default: {  // P_RDN
-          const unsigned cb = (unsigned)cv.n * G.rc_i, sbb = (unsigned)cv.n * G.rs_i;
-          mbar_arrive_expect_tx(&full[slot], (unsigned)G.K * (cb + sbb));
-          uint8_t* dsb = dst + (size_t)G.K * G.rrd * G.rc_i;
-          for (int k = 0; k < G.K; ++k) {
-            const uint8_t* base = L.experts + (size_t)eidx[k] * L.expert_stride + 2 * G.q_gu;
-            stage_rows(dst + (size_t)k * G.rrd * G.rc_i, base + (size_t)cv.r0 * G.rc_i, cb,
-                       &full[slot]);
-            stage_rows(dsb + (size_t)k * G.rrd * G.rs_i,
-                       base + (size_t)G.H * G.rc_i + (size_t)cv.r0 * G.rs_i, sbb, &full[slot]);
-          }
-          break;
+        break;
+      }
+    }
+    sm->issued = i + 1;
+  }
+  // never leave the CTA with bulk copies in flight: wait for the last copies of every stage
+  if (i < n_local) {
+    const uint64_t deadline = global_ns() + 100000000ull;
+    const unsigned first = i > NS ? i - NS : 0u;
+    for (unsigned j = first; j < i; ++j) {
+      const int s = (int)(j % NS);
+      while (!mbar_try_wait(&full[s], (j / NS) & 1u)) {
+        if (global_ns() > deadline) {
+          atomicCAS(P.s.err, 0, DE_TIMEOUT_DRAIN);
+          return;
         }
       }
-      sm->issued = it + 1;
     }
-    __syncwarp();
   }
-  if (lane == 0) sm->prod_done = 1;
 }
 
 // ------------------------------------------------------------------------------------------
-// signal warp: move epilogue results to global memory, publish completions, top-K
+// top-K (stager warp)
 // ------------------------------------------------------------------------------------------
 // Order-preserving 64-bit key of a binary64 value (larger value <=> larger unsigned key).
 __device__ __forceinline__ unsigned long long dkey(double d) {
@@ -350,6 +427,10 @@ __device__ __forceinline__ unsigned long long pkey(double l, int e) {
 __device__ __forceinline__ double dkey_inv(unsigned long long k) {
   const unsigned long long b = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
   return __longlong_as_double((long long)b);
+}
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
 }
 
 // Sort 16 keys in descending order (bitonic network: 80 independent compare-exchanges in 10
@@ -374,35 +455,34 @@ __device__ __forceinline__ void sort16_desc(unsigned long long (&k)[16]) {
   }
 }
 
+// logit of expert e: the sum of its column-segment partials, in segment order
+__device__ __forceinline__ double unit_logit(const Geo& G, const double* lg, int e) {
+  double a = 0.0;
+  for (int s = 0; s < G.rseg; ++s) a += __ldcg(lg + (size_t)s * G.nr + e);
+  return a;
+}
+
 // Top-K of the unit's logits by one warp. Every lane sorts its 16 packed keys; passes over
 // more than 512 experts keep each lane's best 16 by a bitonic merge. Then K rounds of a warp
 // maximum over the lanes' heads (two 32-bit reductions), the winning lane dropping its head.
 // w_k = exp(l_k - l_max) / sum_sel exp(l_j - l_max): the softmax over all experts followed by
 // renormalisation over the selected ones, where the full softmax denominator cancels; the
 // logits come back from the keys with 40 significant bits.
-__device__ __noinline__ void topk_warp(const Prog& P, const Geo& G, int u, int slot,
-                                       const float* bias, int* idx_out, float* w_out,
-                                       Smem* sm) {
+__device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int* rt_e,
+                          float* rt_w, int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
-  const double* lg = P.s.logits + (size_t)slot * G.nr;
   constexpr int kPer = 16;
   unsigned long long best[kPer];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) best[i] = 0ull;
   for (int e0 = 0; e0 < G.E; e0 += 32 * kPer) {
-    double lv[kPer];
-    float bv[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = min(e0 + lane + 32 * i, G.E - 1);
-      lv[i] = __ldcg(lg + e);
-      bv[i] = bias ? __ldcg(bias + e) : 0.f;
-    }
     unsigned long long key[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int e = e0 + lane + 32 * i;
-      key[i] = e < G.E ? pkey(lv[i] + (double)bv[i], e) : 0ull;
+      const int ec = min(e, G.E - 1);
+      const double l = unit_logit(G, lg, ec) + (bias ? (double)__ldcg(bias + ec) : 0.0);
+      key[i] = e < G.E ? pkey(l, e) : 0ull;
     }
     sort16_desc(key);
     if (e0 == 0) {
@@ -412,11 +492,11 @@ __device__ __noinline__ void topk_warp(const Prog& P, const Geo& G, int u, int s
       // both lists sorted descending: best[i] vs key[15-i] keeps the 16 largest as a bitonic
       // sequence, which one more sort puts in order
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) best[i] = best[i] > key[kPer - 1 - i] ? best[i] : key[kPer - 1 - i];
+      for (int i = 0; i < kPer; ++i) best[i] = umax64(best[i], key[kPer - 1 - i]);
       sort16_desc(best);
     }
   }
-  int sel_e = 0;             // lane k < K ends up holding winner k
+  int sel_e = 0;  // lane k < K ends up holding winner k
   unsigned long long sel_k = 0ull;
 #pragma unroll
   for (int k = 0; k < kMaxK; ++k) {
@@ -437,7 +517,6 @@ __device__ __noinline__ void topk_warp(const Prog& P, const Geo& G, int u, int s
       }
     }
   }
-  // weights on lanes 0..K-1
   const double l0 = dkey_inv(__shfl_sync(0xffffffffu, sel_k, 0) & ~0x1FFFull);
   const bool mine = lane < G.K;
   const float ex = mine ? expf((float)(dkey_inv(sel_k & ~0x1FFFull) - l0)) : 0.f;
@@ -447,143 +526,147 @@ __device__ __noinline__ void topk_warp(const Prog& P, const Geo& G, int u, int s
   if (mine) {
     const int e = min(max(sel_e, 0), G.E - 1);  // NaN logits must not make an address
     const float wk = __fdividef(ex, den);
-    sm->rt_e[u & 1][lane] = e;
-    sm->rt_w[u & 1][lane] = wk;
+    rt_e[lane] = e;
+    rt_w[lane] = wk;
     if (idx_out) idx_out[lane] = e;
     if (w_out) w_out[lane] = wk;
   }
   __syncwarp();
 }
 
-// Sum of virtual row vr (wave w = vr / Pn, row-lane p = vr % Pn) from a reduction slot.
-__device__ __forceinline__ float slot_row_sum(const float* part, int vr, int sp, int Pn) {
-  const int p = vr % Pn, w = vr / Pn;
-  if (sp >= 32) {
-    const int nw = sp / 32;
-    float a = 0.f;
-    for (int i = 0; i < nw; ++i) a += part[(p * nw + i) * kMaxW + w];
-    return a;
-  }
-  return part[p * kMaxW + w];
+// ------------------------------------------------------------------------------------------
+// stager warp: per unit, x in, routing decision, down input
+// ------------------------------------------------------------------------------------------
+// Position of float4 number i of 32-column slice t in a transformed vector: swizzled so that
+// the 8 lanes of a quarter-warp reading "float4 i of their own slices" hit distinct banks.
+__device__ __forceinline__ int xpos(int t, int i) { return 32 * t + 4 * (i ^ (t & 7)); }
+
+// x' transform of 4 consecutive values (c a multiple of 4) into the form the slice kernels
+// read: 4-bit pairs (x0, x1/16 - x0); 2-bit quads (x0, x1/4 - x0, x2/16 - x1/4, x3/64 - x2/16).
+__device__ __forceinline__ float4 xform(float4 v, int bits) {
+  if (bits == 4) return make_float4(v.x, v.y * 0.0625f - v.x, v.z, v.w * 0.0625f - v.z);
+  return make_float4(v.x, v.y * 0.25f - v.x, v.z * 0.0625f - v.y * 0.25f,
+                     v.w * 0.015625f - v.z * 0.0625f);
 }
 
-// The signal warp finishes every chunk of its CTA in order: it waits for the eight consumer
-// warps' partials, sums them across warps, applies the epilogue (logit store; SwiGLU;
-// residual/combine), stores the results, frees the slot, and publishes each run of same-
-// (unit, phase) chunks with one gpu-scope fence and one reduction on the phase counter.
-__device__ void signaller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
+// Bring `bytes` from global memory (written by other CTAs or by the caller) into shared
+// memory with one bulk copy and wait for it.
+__device__ __forceinline__ bool stage_in(const Prog& P, Smem* sm, void* dst, const void* src,
+                                         unsigned bytes, unsigned& xphase) {
+  if ((threadIdx.x & 31) == 0) {
+    fence_proxy_async();  // order earlier generic accesses before the async-proxy copy
+    mbar_arrive_expect_tx(&sm->xbar, bytes);
+    tma_load_1d(dst, src, bytes, &sm->xbar);
+  }
+  const bool ok = warp_wait_mbar(P, sm, &sm->xbar, xphase, DE_TIMEOUT_DEP);
+  xphase ^= 1u;
+  return ok;
+}
+
+// Transform nsl slices of raw values in `raw` (linear layout) into `xt` (swizzled) and their
+// sums into `sx`; slice t is scaled by scale_of(t) first (and written back to `raw` when
+// asked). raw and xt may be the same array: a slice is read whole before it is written.
+template <typename ScaleOf>
+__device__ __forceinline__ void transform_slices(float* raw, float* xt, float* sx, int nsl,
+                                                 int bits, ScaleOf scale_of,
+                                                 bool write_back_raw) {
   const int lane = threadIdx.x & 31;
-  float* boxes = reinterpret_cast<float*>(smem + G.o_box);
-  unsigned run_n = 0;
-  int cur_u = -1;
-  UnitView uv;
-  for (ChunkIter ci(P, G); ci.valid(); ci.next()) {
-    const unsigned it = ci.it;
-    // wait until all consumer warps have delivered chunk `it`
-    int ok = 1;
-    if (lane == 0) {
-      const unsigned want = (it + 1) * kConsumerWarps;
-      if ((int)(ld_acquire_cta_smem(&sm->done_count) - want) < 0) {
-        const uint64_t deadline = global_ns() + P.wait_ns;
-        for (unsigned k = 0;; ++k) {
-          if ((int)(ld_acquire_cta_smem(&sm->done_count) - want) >= 0) break;
-          if (sm->abort || sm->cons_done) {
-            __threadfence_block();
-            ok = !sm->abort && (int)(ld_acquire_cta_smem(&sm->done_count) - want) >= 0;
-            break;
-          }
-          if ((k & 63) == 63 && global_ns() > deadline) {
-            raise_error(P, sm, DE_TIMEOUT_DEP);
-            ok = 0;
-            break;
-          }
-          __nanosleep(20);
-        }
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) break;
-    const ChunkView cv = ci.view(G);
-    if (cv.u != cur_u) {
-      cur_u = cv.u;
-      uv = unit_view(P, G, cv.u);
-    }
-    const float* part = boxes + (size_t)(it % kBoxes) * G.box_floats;
-    const float* base = part + G.red_part;
-    float sq = 0.f;
-    for (int r = lane; r < cv.n; r += 32) {
-      switch (cv.phase) {
-        case P_ROUTER: {
-          const double* pd = reinterpret_cast<const double*>(part);
-          double a = 0.0;
-          for (int w = 0; w < kConsumerWarps; ++w) a += pd[w * G.rr + r];
-          P.s.logits[(size_t)uv.slot * G.nr + cv.r0 + r] = a;
-          break;
-        }
-        case P_SGU:
-        case P_RGU: {
-          const float a = slot_row_sum(part, r, G.sp_h, G.p_h);
-          const float u = slot_row_sum(part, G.rcg + r, G.sp_h, G.p_h);
-          const float h = __fdividef(a, 1.f + __expf(-a)) * u;  // SwiGLU: SiLU(gate) * up
-          if (cv.phase == P_SGU)
-            P.s.hs[(size_t)uv.slot * G.I + cv.r0 + r] = h;
-          else
-            P.s.hk[((size_t)uv.slot * G.K + cv.k) * G.I + cv.r0 + r] = h;
-          break;
-        }
-        default: {
-          const bool routed = cv.phase == P_RDN;
-          const float o = base[r] + slot_row_sum(part, r, routed ? G.sp_d : G.sp_i,
-                                                 routed ? G.p_d : G.p_i);
-          uv.out[cv.r0 + r] = o;
-          sq += o * o;
-        }
-      }
-    }
-    const bool final_out = cv.phase == P_RDN || (cv.phase == P_SDN && !G.routed_on);
-    if (final_out && P.mode == MODE_STACK) {
+  for (int t = lane; t < nsl; t += 32) {
+    const float f = scale_of(t);
+    float4 v[8];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) atomicAdd(P.s.normsq + cv.u, sq);
+    for (int i = 0; i < 8; ++i) {  // v[i] = logical float4 q = i ^ (t & 7): distinct banks
+      const int q = i ^ (t & 7);
+      v[i] = *reinterpret_cast<const float4*>(raw + 32 * t + 4 * q);
+      v[i].x *= f; v[i].y *= f; v[i].z *= f; v[i].w *= f;
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    if (write_back_raw) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4*>(raw + 32 * t + 4 * (i ^ (t & 7))) = v[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)  // logical q = i ^ (t & 7) belongs at xpos(t, q) = 32t + 4i
+      *reinterpret_cast<float4*>(xt + 32 * t + 4 * i) = xform(v[i], bits);
+    sx[t] = s;
+  }
+}
+
+__device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
+  const int lane = threadIdx.x & 31;
+  float* XA = reinterpret_cast<float*>(smem + G.o_xa);
+  float* SXA = reinterpret_cast<float*>(smem + G.o_sxa);
+  float* XG = reinterpret_cast<float*>(smem + G.o_xg);
+  float* SXG = reinterpret_cast<float*>(smem + G.o_sxg);
+  const int fcl = final_class(G);
+  const unsigned ntot = (unsigned)G.off[K_COUNT];
+  const bool gu_on = G.shared_on || G.routed_on;
+  unsigned xphase = 0;
+  for (int u = 0; u < P.n_units; ++u) {
+    const UnitView uv = unit_view(P, G, u);
+    const bool owner = ((unsigned long long)u * ntot) % gridDim.x == blockIdx.x;
+    // ---- x(u): needs unit u-1 complete (its output is this input, its buffers are free)
+    if (u > 0 && !warp_wait_flag(P, sm, fcl, (unsigned)u, DE_TIMEOUT_DEP)) break;
+    float f = 1.f;
+    if (uv.norm) f = rsqrtf(__ldcg(P.s.normsq + (u - 1)) / (float)G.H + P.eps);
+    if (!stage_in(P, sm, XA, uv.xin, 4u * (unsigned)G.H, xphase)) break;
+    if (owner && uv.h_trace)
+      for (int c = lane * 4; c < G.H; c += 128)
+        *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XA + c);
+    if (gu_on) {
+      transform_slices(XA, XG, SXG, G.H / 32, G.bits, [&](int) { return f; },
+                       G.route_on && uv.norm);
+    } else if (uv.norm) {
+      for (int c = lane * 4; c < G.H; c += 128) {
+        float4 v = *reinterpret_cast<float4*>(XA + c);
+        v.x *= f; v.y *= f; v.z *= f; v.w *= f;
+        *reinterpret_cast<float4*>(XA + c) = v;
+      }
     }
     __syncwarp();
-    if (lane == 0) sm->sig_done = it + 1;  // the slot may be reused
-    ++run_n;
-    // Publish when this CTA's run of (unit, phase) ends: the next chunk of the schedule
-    // belongs to another unit or phase, or there is none.
-    ChunkIter nx = ci;
-    nx.next();
-    bool run_end = !nx.valid();
-    if (!run_end) {
-      const ChunkView nv = nx.view(G);
-      run_end = nv.u != cv.u || nv.phase != cv.phase;
-    }
-    if (run_end) {
-      fence_acq_rel_gpu();  // every lane: its stores come first
+    if (lane == 0) st_release_cta_smem(&sm->x_ready, (unsigned)(u + 1));
+    // ---- routing decision: needs every router chunk of unit u
+    float sigma = 1.f;
+    if (G.route_on) {
+      if (!warp_wait_flag(P, sm, CL_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) break;
+      const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
+      if (G.gate_on)  // sigma(g . x): the shared-gate row is router row E
+        sigma = (float)(1.0 / (1.0 + exp(-unit_logit(G, lg, G.E))));
+      topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
+                owner ? uv.w_out : nullptr);
       __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        const unsigned old = atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cv.phase), run_n);
-        last = old + run_n == (unsigned)(cv.u + 1) * (unsigned)G.n[cv.phase];
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        // this CTA completed the phase for the unit: tell every CTA through its own flag line
-        if (cv.phase == P_ROUTER && !G.routed_on)  // routing-only launches: outputs from here
-          topk_warp(P, G, cv.u, uv.slot, uv.bias, uv.idx_out, uv.w_out, sm);
-        if (!(cv.phase == P_ROUTER && (P.debug & 1))) {
-          fence_acq_rel_gpu();
-          for (int c = lane; c < (int)gridDim.x; c += 32)
-            P.s.flags[c * F_WORDS + cv.phase] = (unsigned)(cv.u + 1);
-        }
-      }
-      run_n = 0;
+      if (lane == 0) st_release_cta_smem(&sm->rt_ready, (unsigned)(u + 1));
+    }
+    // ---- down input [sigma*h_s | w_0*h_0 | ...]: needs every gate/up chunk of unit u
+    if (G.nseg > 0) {
+      if (!warp_wait_flag(P, sm, CL_GU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
+      bool ok = true;
+      if (G.shared_on)
+        ok = stage_in(P, sm, XA, P.s.hs + (size_t)uv.slot * G.I, 4u * (unsigned)G.I, xphase);
+      if (ok && G.routed_on)
+        ok = stage_in(P, sm, XA + (size_t)G.shared_on * G.I,
+                      P.s.hk + (size_t)uv.slot * G.K * G.I, 4u * (unsigned)(G.K * G.I), xphase);
+      if (!ok) break;
+      const int spseg = G.I / 32;
+      const float* rw = sm->rt_w[u & 1];
+      transform_slices(
+          XA, XA, SXA, G.nseg * spseg, G.bits,
+          [&](int t) {
+            const int s = t / spseg;
+            return (G.shared_on && s == 0) ? sigma : rw[s - G.shared_on];
+          },
+          false);
+      __syncwarp();
+      if (lane == 0) st_release_cta_smem(&sm->xd_ready, (unsigned)(u + 1));
     }
   }
 }
 
 // ------------------------------------------------------------------------------------------
-// dequantising dot products of W rows with one thread's 32-column slice
+// dequantising dot products: W rows x one 32-column slice
 // ------------------------------------------------------------------------------------------
 // One byte of codes becomes the binary32 32768 + byte (exponent 15, byte in mantissa bits
 // 8..15); clearing the low code(s) gives 32768 + the high part. Subtracting 32768 is exact.
@@ -591,39 +674,33 @@ __device__ __forceinline__ uint32_t magic_byte(uint32_t word, int k) {
   return __byte_perm(word, 0x47000000u, 0x7604u | ((uint32_t)k << 4));
 }
 
-// v[w] = s_w * sum(q x) + z_w * sum(x) over the slice, for the W rows vr = p + w*P; all W
-// rows are loaded first and unpacked in lock step so their instruction streams interleave.
-// Rows that are not valid read a clamped (in-stage) address and are returned as 0.
+// acc[w] += s_w * sum(q x) + z_w * sum(x) over the slice, for W rows whose codes start at
+// stage + coff[w] and whose scale/bias word is at stage + soff[w]; rows with ok[w] false add
+// 0 (their offsets must still point inside the stage).
 template <int BITS, int W>
-__device__ __forceinline__ void qrows(const uint8_t* slot, int p, int P, bool s_ok,
-                                      unsigned a_row, unsigned a_slice, unsigned b_base,
-                                      unsigned b_row, unsigned b_slice, int n, int half_rows,
-                                      int vmax, const float (&xq)[32], float sx, float (&v)[W]) {
+__device__ __forceinline__ void qslice(const uint8_t* stage, const unsigned (&coff)[W],
+                                       const unsigned (&soff)[W], const bool (&ok)[W],
+                                       const float (&xq)[32], float sx, float* acc) {
   constexpr int kWords = BITS == 4 ? 4 : 2;
   uint32_t q[W][kWords];
   uint32_t sbw[W];
-  bool ok[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) {
-    const int vr = p + w * P;
-    ok[w] = s_ok && (half_rows > 0 ? (vr < half_rows ? vr < n : (vr - half_rows) < n) : vr < n);
-    const int vc = min(vr, vmax);
-    const uint8_t* ca = slot + a_slice + (size_t)vc * a_row;
     if constexpr (BITS == 4) {
-      const uint4 t = *reinterpret_cast<const uint4*>(ca);
+      const uint4 t = *reinterpret_cast<const uint4*>(stage + coff[w]);
       q[w][0] = t.x; q[w][1] = t.y; q[w][2] = t.z; q[w][3] = t.w;
     } else {
-      const uint2 t = *reinterpret_cast<const uint2*>(ca);
+      const uint2 t = *reinterpret_cast<const uint2*>(stage + coff[w]);
       q[w][0] = t.x; q[w][1] = t.y;
     }
-    sbw[w] = *reinterpret_cast<const uint32_t*>(slot + b_base + b_slice + (size_t)vc * b_row);
+    sbw[w] = *reinterpret_cast<const uint32_t*>(stage + soff[w]);
   }
   const float2 m = make_float2(-32768.f, -32768.f);
-  float2 acc0[W], acc1[W];
+  float2 a0[W], a1[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) {
-    acc0[w] = make_float2(0.f, 0.f);
-    acc1[w] = make_float2(0.f, 0.f);
+    a0[w] = make_float2(0.f, 0.f);
+    a1[w] = make_float2(0.f, 0.f);
   }
 #pragma unroll
   for (int wi = 0; wi < kWords; ++wi) {
@@ -636,11 +713,12 @@ __device__ __forceinline__ void qrows(const uint8_t* slot, int p, int P, bool s_
 #pragma unroll
         for (int w = 0; w < W; ++w) {
           const uint32_t t = magic_byte(q[w][wi], k);
-          const float2 f = __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFF0FFu)), m);
+          const float2 f =
+              __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFF0FFu)), m);
           if (b & 1)
-            acc1[w] = __ffma2_rn(f, xv, acc1[w]);
+            a1[w] = __ffma2_rn(f, xv, a1[w]);
           else
-            acc0[w] = __ffma2_rn(f, xv, acc0[w]);
+            a0[w] = __ffma2_rn(f, xv, a0[w]);
         }
       } else {
         // (c0+4c1+16c2+64c3, 4c1+16c2+64c3) and (16c2+64c3, 64c3)
@@ -649,10 +727,12 @@ __device__ __forceinline__ void qrows(const uint8_t* slot, int p, int P, bool s_
 #pragma unroll
         for (int w = 0; w < W; ++w) {
           const uint32_t t = magic_byte(q[w][wi], k);
-          const float2 f01 = __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFFCFFu)), m);
-          const float2 f23 = __fadd2_rn(make_float2(__uint_as_float(t & 0xFFFFF0FFu), __uint_as_float(t & 0xFFFFC0FFu)), m);
-          acc0[w] = __ffma2_rn(f01, xa, acc0[w]);
-          acc1[w] = __ffma2_rn(f23, xb, acc1[w]);
+          const float2 f01 =
+              __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFFCFFu)), m);
+          const float2 f23 = __fadd2_rn(
+              make_float2(__uint_as_float(t & 0xFFFFF0FFu), __uint_as_float(t & 0xFFFFC0FFu)), m);
+          a0[w] = __ffma2_rn(f01, xa, a0[w]);
+          a1[w] = __ffma2_rn(f23, xb, a1[w]);
         }
       }
     }
@@ -661,8 +741,8 @@ __device__ __forceinline__ void qrows(const uint8_t* slot, int p, int P, bool s_
   for (int w = 0; w < W; ++w) {
     const float s = __uint_as_float(sbw[w] << 16);
     const float z = __uint_as_float(sbw[w] & 0xFFFF0000u);
-    const float qx = (acc0[w].x + acc0[w].y) + (acc1[w].x + acc1[w].y);
-    v[w] = ok[w] ? fmaf(s, qx, z * sx) : 0.f;
+    const float qx = (a0[w].x + a0[w].y) + (a1[w].x + a1[w].y);
+    acc[w] += ok[w] ? fmaf(s, qx, z * sx) : 0.f;
   }
 }
 
@@ -701,392 +781,225 @@ __device__ __forceinline__ void reduce_rows(float (&v)[W], int lane_in_seg, int 
   }
 }
 
-// x' transform of a vector into the layout the slice kernels read (see qrows): 4-bit pairs
-// (x0, x1/16 - x0); 2-bit quads (x0, x1/4 - x0, x2/16 - x1/4, x3/64 - x2/16).
-__device__ __forceinline__ void transform_store4(float* xq, int c, float v0, float v1, float v2,
-                                                 float v3, int bits) {
-  float4 o;
-  if (bits == 4)
-    o = make_float4(v0, v1 * 0.0625f - v0, v2, v3 * 0.0625f - v2);
-  else
-    o = make_float4(v0, v1 * 0.25f - v0, v2 * 0.0625f - v1 * 0.25f, v3 * 0.015625f - v2 * 0.0625f);
-  *reinterpret_cast<float4*>(xq + c) = o;
+// Where a chunk's rows live in its stage.
+struct RowGeom {
+  unsigned rc, rs;        // row strides (codes, sb) inside a segment
+  unsigned seg_c, seg_s;  // segment strides (codes, sb)
+  unsigned sb0;           // offset of the sb area
+  int spseg;              // slices per segment
+};
+
+// A chunk's rows x slices on one warp: rows rho = lane_p + P*i (i < NRL), slices
+// t = lane_s + S*j; rows are processed in lock-step groups of GW (3 or 4) per slice. The
+// reduced value of row rho ends in red[(rho % P) * kRowsPerLane + rho / P].
+template <int BITS, int NRL, typename Valid>
+__device__ __forceinline__ void dot_chunk(const uint8_t* stage, const LaneMap& M,
+                                          const RowGeom& RG, int nrows, Valid valid,
+                                          const float* X, const float* SX, float* red) {
+  constexpr int NRLP = NRL <= 4 ? 4 : 8;         // padded to a power of two for the butterfly
+  constexpr int GW = (NRL % 4 == 0) ? 4 : 3;     // rows per lock-step group
+  const int lane = threadIdx.x & 31;
+  const int lane_s = lane & (M.S - 1), lane_p = lane / M.S;
+  constexpr unsigned cb = BITS == 4 ? 16u : 8u;
+  float acc[NRLP];
+#pragma unroll
+  for (int i = 0; i < NRLP; ++i) acc[i] = 0.f;
+  const int nj = (M.nsl + M.S - 1) / M.S;
+  for (int j = 0; j < nj; ++j) {
+    const int t = lane_s + M.S * j;
+    const bool tok = t < M.nsl;
+    const int tc = tok ? t : M.nsl - 1;
+    float xq[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 a = *reinterpret_cast<const float4*>(X + xpos(tc, i));
+      xq[4 * i] = a.x; xq[4 * i + 1] = a.y; xq[4 * i + 2] = a.z; xq[4 * i + 3] = a.w;
+    }
+    const float sx = SX[tc];
+    const int seg = tc / RG.spseg, loc = tc - seg * RG.spseg;
+    const unsigned cbase = (unsigned)seg * RG.seg_c + (unsigned)loc * cb;
+    const unsigned sbase = RG.sb0 + (unsigned)seg * RG.seg_s + (unsigned)(loc >> 1) * 4u;
+#pragma unroll
+    for (int g = 0; g < NRL; g += GW) {
+      if (g == 0 || M.P * g < nrows) {  // some lane has rows in this group
+        unsigned coff[GW], soff[GW];
+        bool ok[GW];
+#pragma unroll
+        for (int w = 0; w < GW; ++w) {
+          const int rho = lane_p + M.P * (g + w);
+          ok[w] = tok && valid(rho);
+          const unsigned rr = ok[w] ? (unsigned)rho : 0u;
+          coff[w] = cbase + rr * RG.rc;
+          soff[w] = sbase + rr * RG.rs;
+        }
+        qslice<BITS, GW>(stage, coff, soff, ok, xq, sx, acc + g);
+      }
+    }
+  }
+  reduce_rows<NRLP>(acc, lane_s, M.S, red + lane_p * kRowsPerLane);
+}
+
+__device__ __forceinline__ float red_row(const float* red, const LaneMap& M, int rho) {
+  return red[(rho % M.P) * kRowsPerLane + rho / M.P];
 }
 
 // ------------------------------------------------------------------------------------------
-// consumers
+// consumer warps
 // ------------------------------------------------------------------------------------------
-struct Map {  // one thread's place in a virtual-row layout: row-lane p, slice s (clamped sc)
-  int p, s, sc;
-  bool ok;
-};
-
-__device__ __forceinline__ Map make_map(int sp, int Pn, int sl) {
-  Map m;
-  m.p = ctid() / sp;
-  m.s = ctid() - m.p * sp;
-  m.ok = m.p < Pn && m.s < sl;
-  m.sc = min(m.s, sl - 1);
-  return m;
+__device__ __forceinline__ void release_stage(uint64_t* empty) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
 }
 
-struct Consumer {
-  const Prog& P;
-  const Geo& G;
-  uint8_t* smem;
-  Smem* sm;
-  float* XR;
-  float* XG;
-  float* SXG;
-  float* XS;
-  float* SXS;
-  float* XD;
-  float* SXD;
-  float* boxes;
-  Map mgu, msd, mrd;
-  int x_unit = -1, xs_unit = -1, xd_unit = -1;
-  int tag_unit = -1, tag_buf = -1;
-  float xq[32];
-  float sx = 0.f;
-
-  __device__ Consumer(const Prog& P_, const Geo& G_, uint8_t* smem_, Smem* sm_)
-      : P(P_), G(G_), smem(smem_), sm(sm_) {
-    XR = reinterpret_cast<float*>(smem + G.o_xr);
-    XG = reinterpret_cast<float*>(smem + G.o_xg);
-    SXG = reinterpret_cast<float*>(smem + G.o_sxg);
-    XS = reinterpret_cast<float*>(smem + G.o_xs);
-    SXS = reinterpret_cast<float*>(smem + G.o_sxs);
-    XD = reinterpret_cast<float*>(smem + G.o_xd);
-    SXD = reinterpret_cast<float*>(smem + G.o_sxd);
-    boxes = reinterpret_cast<float*>(smem + G.o_box);
-    mgu = make_map(G.sp_h, G.p_h, G.sl_h);
-    msd = make_map(G.sp_i, G.p_i, G.sl_i);
-    mrd = make_map(G.sp_d, G.p_d, G.sl_d);
-  }
-
-  __device__ __forceinline__ bool wait_unit_done(int u) {
-    return consumer_wait(P, sm, final_phase(G), (unsigned)(u + 1), DE_TIMEOUT_DEP);
-  }
-
-  // slice sums of a vector in shared memory (32 columns per slice), bank-conflict free
-  __device__ __forceinline__ void slice_sums(const float* x, float* sxo, int nsl) {
-    for (int s = ctid(); s < nsl; s += kConsumers) {
-      float a = 0.f;
-      for (int i = 0; i < 32; ++i) a += x[s * 32 + ((i + s) & 31)];
-      sxo[s] = a;
+// router rows r0..r0+n-1, columns seg*rcols .. +rcols: binary64 sums of fp32 products
+__device__ __forceinline__ void router_chunk(const Prog& P, const Geo& G, const Chunk& cv,
+                                             const uint8_t* stage, uint64_t* empty,
+                                             const float* XR) {
+  const int lane = threadIdx.x & 31;
+  const float4* xr = reinterpret_cast<const float4*>(XR + (size_t)cv.seg * G.rcols);
+  const int nf = G.rcols / 4;
+  double* lg = P.s.logits + ((size_t)(cv.u & 1) * G.rseg + cv.seg) * G.nr + cv.r0;
+  double res = 0.0;
+  for (int r = 0; r < cv.n; ++r) {
+    const float4* wr = reinterpret_cast<const float4*>(stage) + (size_t)r * nf;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    for (int f = lane; f < nf; f += 32) {
+      const float4 w = wr[f], x = xr[f];
+      a0 = fma((double)w.x, (double)x.x, a0);
+      a1 = fma((double)w.y, (double)x.y, a1);
+      a2 = fma((double)w.z, (double)x.z, a2);
+      a3 = fma((double)w.w, (double)x.w, a3);
     }
-  }
-
-  // x of unit u: raw in XR (router), transformed in XG + slice sums (gate/up)
-  __device__ __forceinline__ bool ensure_x(int u, const UnitView& uv) {
-    if (x_unit == u) return true;
-    if (u > 0 && !wait_unit_done(u - 1)) return false;
-    float f = 1.f;
-    if (uv.norm) f = rsqrtf(__ldcg(P.s.normsq + (u - 1)) / (float)G.H + P.eps);
-    for (int c = ctid() * 4; c < G.H; c += kConsumers * 4) {
-      const float4 a = ldcg4(uv.xin + c);
-      const float v0 = a.x * f, v1 = a.y * f, v2 = a.z * f, v3 = a.w * f;
-      *reinterpret_cast<float4*>(XR + c) = make_float4(v0, v1, v2, v3);
-      transform_store4(XG, c, v0, v1, v2, v3, G.bits);
-    }
-    consumer_sync();
-    slice_sums(XR, SXG, G.sl_h);
-    consumer_sync();
-    x_unit = u;
-    return true;
-  }
-
-  // sigma * h_shared, transformed, for the shared-expert down rows
-  __device__ __forceinline__ bool ensure_xs(int u, const UnitView& uv) {
-    if (xs_unit == u) return true;
-    if (!consumer_wait(P, sm, P_SGU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) return false;
-    float sig = 1.f;
-    if (G.gate_on) {  // sigma(g . x): the shared-gate row is the last router row
-      if (!consumer_wait(P, sm, P_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_DEP)) return false;
-      sig = (float)(1.0 / (1.0 + exp(-__ldcg(P.s.logits + (size_t)uv.slot * G.nr + G.E))));
-    }
-    const float* hs = P.s.hs + (size_t)uv.slot * G.I;
-    float* raw = XD;  // XD is rebuilt before its next use in this unit
-    for (int c = ctid() * 4; c < G.I; c += kConsumers * 4) {
-      const float4 a = ldcg4(hs + c);
-      const float v0 = sig * a.x, v1 = sig * a.y, v2 = sig * a.z, v3 = sig * a.w;
-      *reinterpret_cast<float4*>(raw + c) = make_float4(v0, v1, v2, v3);
-      transform_store4(XS, c, v0, v1, v2, v3, G.bits);
-    }
-    consumer_sync();
-    slice_sums(raw, SXS, G.sl_i);
-    xd_unit = -1;
-    consumer_sync();
-    xs_unit = u;
-    return true;
-  }
-
-  // w_k * h_k of the routed experts, transformed, for the routed down rows
-  __device__ __forceinline__ bool ensure_xd(int u, const UnitView& uv) {
-    if (xd_unit == u) return true;
-    if (!consumer_wait(P, sm, P_RGU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) return false;
-    if (G.shared_on && !consumer_wait(P, sm, P_SDN, (unsigned)(u + 1), DE_TIMEOUT_DEP))
-      return false;
-    const float* hk = P.s.hk + (size_t)uv.slot * G.K * G.I;
-    const int KI = G.K * G.I;
-    float* raw = XR;  // XR (the router's x) is no longer needed in this unit
-    for (int c = ctid() * 4; c < KI; c += kConsumers * 4) {
-      const float wk = sm->rt_w[u & 1][c / G.I];
-      const float4 a = ldcg4(hk + c);
-      const float v0 = wk * a.x, v1 = wk * a.y, v2 = wk * a.z, v3 = wk * a.w;
-      if (KI <= G.H) *reinterpret_cast<float4*>(raw + c) = make_float4(v0, v1, v2, v3);
-      transform_store4(XD, c, v0, v1, v2, v3, G.bits);
-    }
-    consumer_sync();
-    if (KI <= G.H) {
-      slice_sums(raw, SXD, G.sl_d);
-    } else {
-      for (int s = ctid(); s < G.sl_d; s += kConsumers) {
-        const float wk = sm->rt_w[u & 1][(s * 32) / G.I];
-        float a = 0.f;
-        for (int i = 0; i < 32; ++i) a += wk * __ldcg(hk + s * 32 + i);
-        SXD[s] = a;
-      }
-    }
-    if (KI <= G.H) x_unit = -1;  // XR was overwritten
-    consumer_sync();
-    xd_unit = u;
-    return true;
-  }
-
-  __device__ __forceinline__ void load_xq(int unit, int buf, const float* X, const float* SX,
-                                          const Map& m) {
-    if (tag_unit == unit && tag_buf == buf) return;
-    tag_unit = unit;
-    tag_buf = buf;
-    if (m.ok) {
-      const float4* src = reinterpret_cast<const float4*>(X + m.s * 32);
+    double a = (a0 + a1) + (a2 + a3);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 a = src[i];
-        xq[4 * i] = a.x;
-        xq[4 * i + 1] = a.y;
-        xq[4 * i + 2] = a.z;
-        xq[4 * i + 3] = a.w;
-      }
-      sx = SX[m.s];
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == (r & 31)) res = a;
+    if ((r & 31) == 31 || r == cv.n - 1) {  // flush up to 32 results, one per lane
+      const int rb = r & ~31;
+      if (lane <= (r & 31)) lg[rb + lane] = res;
     }
   }
+  release_stage(empty);
+}
 
-  // Slot of chunk `it` may be written once the signal warp has finished chunk it - kBoxes.
-  // Each warp checks for itself (no CTA-wide barrier per chunk).
-  __device__ __forceinline__ void wait_slot(unsigned it) {
-    if ((threadIdx.x & 31) == 0 && it >= (unsigned)kBoxes) {
-      const unsigned want = it - kBoxes + 1;
-      if ((int)(sm->sig_done - want) < 0) {
-        const uint64_t deadline = global_ns() + P.wait_ns;
-        for (unsigned k = 0;; ++k) {
-          if ((int)(sm->sig_done - want) >= 0) break;
-          if (sm->abort) break;
-          if ((k & 63) == 63 && global_ns() > deadline) {
-            raise_error(P, sm, DE_TIMEOUT_DEP);
-            break;
-          }
-          __nanosleep(20);
-        }
-      }
-    }
-    __syncwarp();
+template <int BITS, int NRL>
+__device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, const Chunk& cv,
+                                         const uint8_t* stage, uint64_t* empty, const float* XG,
+                                         const float* SXG, float* red) {
+  const int lane = threadIdx.x & 31;
+  RowGeom RG;
+  RG.rc = G.rc_h; RG.rs = G.rs_h; RG.seg_c = 0; RG.seg_s = 0;
+  RG.sb0 = 2u * (unsigned)G.R * G.rc_h;
+  RG.spseg = G.H / 32;
+  const int R = G.R, n = cv.n;
+  dot_chunk<BITS, NRL>(
+      stage, G.gu, RG, 2 * R,
+      [&](int rho) { return rho < 2 * R && (rho < R ? rho : rho - R) < n; }, XG, SXG, red);
+  release_stage(empty);
+  __syncwarp();
+  float* h = cv.kind == K_SGU ? P.s.hs + (size_t)(cv.u & 1) * G.I
+                              : P.s.hk + ((size_t)(cv.u & 1) * G.K + cv.k) * G.I;
+  for (int r = lane; r < n; r += 32) {
+    const float a = red_row(red, G.gu, r);
+    const float b = red_row(red, G.gu, R + r);
+    h[cv.r0 + r] = __fdividef(a, 1.f + __expf(-a)) * b;  // SwiGLU: SiLU(gate) * up
   }
+  __syncwarp();
+}
 
-  // Warp-level reduction of the row partials straight into the chunk's slot.
-  template <int W>
-  __device__ __forceinline__ void reduce_to_slot(float (&v)[W], int sp, unsigned it,
-                                                 float* part) {
-    const int lane = threadIdx.x & 31, warp = (ctid() >> 5);
-    const int width = sp < 32 ? sp : 32;
-    float* dst = sp >= 32 ? part + warp * kMaxW : part + (warp * (32 / sp) + lane / sp) * kMaxW;
-    const int lane_in_seg = sp >= 32 ? lane : (lane % sp);
-    wait_slot(it);
-    reduce_rows<W>(v, lane_in_seg, width, dst);
+template <int BITS, int NRL>
+__device__ __forceinline__ void dn_chunk(const Prog& P, const Geo& G, const Chunk& cv,
+                                         const UnitView& uv, const uint8_t* stage,
+                                         uint64_t* empty, const float* XD, const float* SXD,
+                                         float* red) {
+  const int lane = threadIdx.x & 31;
+  // the residual each output row adds is fetched first so its latency hides behind the dots
+  const float rv = (uv.res && lane < cv.n) ? __ldcg(uv.res + cv.r0 + lane) : 0.f;
+  RowGeom RG;
+  RG.rc = G.rc_i; RG.rs = G.rs_i;
+  RG.seg_c = (unsigned)G.Rd * G.rc_i;
+  RG.seg_s = (unsigned)G.Rd * G.rs_i;
+  RG.sb0 = (unsigned)G.nseg * G.Rd * G.rc_i;
+  RG.spseg = G.I / 32;
+  const int n = cv.n;
+  dot_chunk<BITS, NRL>(stage, G.dn, RG, n, [&](int rho) { return rho < n; }, XD, SXD, red);
+  release_stage(empty);
+  __syncwarp();
+  float sq = 0.f;
+  for (int r = lane; r < n; r += 32) {
+    const float base = r < 32 ? rv : (uv.res ? __ldcg(uv.res + cv.r0 + r) : 0.f);
+    const float o = base + red_row(red, G.dn, r);
+    uv.out[cv.r0 + r] = o;
+    sq += o * o;
   }
-
-  // Epilogue row of this thread for prefetches: rows go round-robin over the warps (row r ->
-  // warp r % 8, lane r / 8) so that no single warp carries them.
-  __device__ __forceinline__ int epi_row() const {
-    return (threadIdx.x & 31) * kConsumerWarps + ((ctid() >> 5));
-  }
-
-  __device__ __forceinline__ void release(uint64_t* empty) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
-  }
-
-  // ---------------------------------------------------------------- router rows
-  __device__ __forceinline__ void router_chunk(const ChunkView& cv, const uint8_t* slot,
-                                               uint64_t* empty, float* part, unsigned it) {
-    const float* rows = reinterpret_cast<const float*>(slot);
-    const int H = G.H, t = ctid(), lane = t & 31, warp = t >> 5;
-    if (lane == 0) wait_slot_lane0(it);
-    __syncwarp();
-    for (int r = 0; r < cv.n; ++r) {
-      double a = 0.0;
-      const float4* wr = reinterpret_cast<const float4*>(rows + (size_t)r * H);
-      const float4* xr = reinterpret_cast<const float4*>(XR);
-      for (int c4 = t; c4 < H / 4; c4 += kConsumers) {
-        const float4 p = wr[c4], b = xr[c4];
-        a = fma((double)p.x, (double)b.x, a);
-        a = fma((double)p.y, (double)b.y, a);
-        a = fma((double)p.z, (double)b.z, a);
-        a = fma((double)p.w, (double)b.w, a);
-      }
+  if (P.mode == MODE_STACK) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) reinterpret_cast<double*>(part)[warp * G.rr + r] = a;
-    }
-    release(empty);
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) atomicAdd(P.s.normsq + cv.u, sq);
   }
+  __syncwarp();
+}
 
-  __device__ __forceinline__ void wait_slot_lane0(unsigned it) {
-    if (it >= (unsigned)kBoxes) {
-      const unsigned want = it - kBoxes + 1;
-      const uint64_t deadline = global_ns() + P.wait_ns;
-      for (unsigned k = 0; (int)(sm->sig_done - want) < 0; ++k) {
-        if (sm->abort) break;
-        if ((k & 63) == 63 && global_ns() > deadline) {
-          raise_error(P, sm, DE_TIMEOUT_DEP);
-          break;
-        }
-        __nanosleep(20);
-      }
-    }
-  }
+// rows per lane -> the compiled variant that covers them (3, 4, 6 or 8 rows)
+__device__ __forceinline__ int nrl_class(int nrl) {
+  return nrl <= 3 ? 3 : (nrl == 4 ? 4 : (nrl <= 6 ? 6 : 8));
+}
 
-  // ---------------------------------------------------------------- gate/up (SwiGLU in the signal warp)
-  template <int BITS, int W>
-  __device__ __forceinline__ void gateup_chunk(const ChunkView& cv, const uint8_t* slot,
-                                               uint64_t* empty, float* part, unsigned it) {
-    load_xq(cv.u, 0, XG, SXG, mgu);
-    float v[W];
-    qrows<BITS, W>(slot, mgu.p, G.p_h, mgu.ok, G.rc_h, (unsigned)mgu.sc * (BITS == 4 ? 16u : 8u),
-                   2u * G.rcg * G.rc_h, G.rs_h, (unsigned)(mgu.sc >> 1) * 4u, cv.n, G.rcg,
-                   2 * G.rcg - 1, xq, sx, v);
-    release(empty);
-    reduce_to_slot<W>(v, G.sp_h, it, part);
+template <int BITS>
+__device__ __forceinline__ void dispatch_dot(const Prog& P, const Geo& G, const Chunk& cv,
+                                             const UnitView& uv, const uint8_t* stage,
+                                             uint64_t* empty, uint8_t* smem, float* red) {
+  if (cv.kind == K_DN) {
+    const float* XD = reinterpret_cast<const float*>(smem + G.o_xa);
+    const float* SXD = reinterpret_cast<const float*>(smem + G.o_sxa);
+    switch (nrl_class(G.dn.nrl)) {
+      case 3: dn_chunk<BITS, 3>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
+      case 4: dn_chunk<BITS, 4>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
+      case 6: dn_chunk<BITS, 6>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
+      default: dn_chunk<BITS, 8>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
+    }
+  } else {
+    const float* XG = reinterpret_cast<const float*>(smem + G.o_xg);
+    const float* SXG = reinterpret_cast<const float*>(smem + G.o_sxg);
+    switch (nrl_class(G.gu.nrl)) {
+      case 3: gu_chunk<BITS, 3>(P, G, cv, stage, empty, XG, SXG, red); break;
+      case 4: gu_chunk<BITS, 4>(P, G, cv, stage, empty, XG, SXG, red); break;
+      case 6: gu_chunk<BITS, 6>(P, G, cv, stage, empty, XG, SXG, red); break;
+      default: gu_chunk<BITS, 8>(P, G, cv, stage, empty, XG, SXG, red); break;
+    }
   }
+}
 
-  // ---------------------------------------------------------------- down (+ base for the combine)
-  template <int BITS, int W>
-  __device__ __forceinline__ void down_chunk(const ChunkView& cv, const UnitView& uv,
-                                             const uint8_t* slot, uint64_t* empty, float* part,
-                                             unsigned it, bool fail) {
-    const bool routed = cv.phase == P_RDN;
-    const Map& m = routed ? mrd : msd;
-    const int sp = routed ? G.sp_d : G.sp_i, Pn = routed ? G.p_d : G.p_i;
-    const int rows = routed ? G.rrd : G.rsd;
-    // the base each output row adds to (residual, or the shared expert's combine) is fetched
-    // now so its latency hides behind the dot products; the signal warp adds it
-    float base[2];
-    const int er = epi_row();
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int r = er + i * kConsumers;
-      base[i] = 0.f;
-      if (r < cv.n && !fail) {
-        const int j = cv.r0 + r;
-        if (routed && G.shared_on)
-          base[i] = __ldcg(uv.out + j);
-        else if (uv.res)
-          base[i] = __ldcg(uv.res + j);
-      }
+__device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, int w) {
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_full);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
+  float* red = reinterpret_cast<float*>(smem + G.o_red) + (size_t)w * 16 * kRowsPerLane;
+  const float* XR = reinterpret_cast<const float*>(smem + G.o_xa);
+  const unsigned NS = (unsigned)G.nstage;
+  const unsigned n_local = local_chunks(P, G);
+  int cur_u = -1;
+  UnitView uv;
+  for (unsigned i = (unsigned)w; i < n_local; i += kConsumerWarps) {
+    const int slot = (int)(i % NS);
+    if (!warp_wait_mbar(P, sm, &full[slot], (i / NS) & 1u, DE_TIMEOUT_FULL)) break;
+    const Chunk cv =
+        chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
+    if (cv.u != cur_u) {
+      cur_u = cv.u;
+      uv = unit_view(P, G, cv.u);
     }
-    unsigned a_slice, b_slice;
-    const unsigned b_base = (unsigned)(routed ? G.K : 1) * rows * G.rc_i;
-    const unsigned cbytes = BITS == 4 ? 16u : 8u;
-    if (routed) {
-      const int k = m.sc / G.sl_i, si = m.sc - k * G.sl_i;
-      a_slice = (unsigned)k * rows * G.rc_i + (unsigned)si * cbytes;
-      b_slice = (unsigned)k * rows * G.rs_i + (unsigned)(si >> 1) * 4u;
-      load_xq(cv.u, 2, XD, SXD, m);
-    } else {
-      a_slice = (unsigned)m.sc * cbytes;
-      b_slice = (unsigned)(m.sc >> 1) * 4u;
-      load_xq(cv.u, 1, XS, SXS, m);
-    }
-    float v[W];
-    qrows<BITS, W>(slot, m.p, Pn, m.ok, G.rc_i, a_slice, b_base, G.rs_i, b_slice, cv.n, 0,
-                   rows - 1, xq, sx, v);
-    release(empty);
-    reduce_to_slot<W>(v, sp, it, part);
-    float* bs = part + G.red_part;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int r = er + i * kConsumers;
-      if (r < cv.n) bs[r] = base[i];
-    }
+    const unsigned* ready = cv.kind == K_DN ? &sm->xd_ready : &sm->x_ready;
+    if (!warp_wait_smem(P, sm, ready, (unsigned)(cv.u + 1), DE_TIMEOUT_DEP)) break;
+    const uint8_t* stage = smem + G.o_ring + (size_t)slot * G.stage_bytes;
+    if (cv.kind == K_ROUTER)
+      router_chunk(P, G, cv, stage, &empty[slot], XR);
+    else if (G.bits == 4)
+      dispatch_dot<4>(P, G, cv, uv, stage, &empty[slot], smem, red);
+    else
+      dispatch_dot<2>(P, G, cv, uv, stage, &empty[slot], smem, red);
+    finish_chunk(P, G, sm, class_of(cv.kind), cv.u);
   }
-
-  template <int BITS>
-  __device__ __forceinline__ void dispatch(const ChunkView& cv, const UnitView& uv,
-                                           const uint8_t* slot, uint64_t* empty, float* part,
-                                           unsigned it, bool fail) {
-    if (cv.phase == P_SGU || cv.phase == P_RGU) {
-      if (G.w_gu == 4)
-        gateup_chunk<BITS, 4>(cv, slot, empty, part, it);
-      else
-        gateup_chunk<BITS, 8>(cv, slot, empty, part, it);
-    } else {
-      down_chunk<BITS, 4>(cv, uv, slot, empty, part, it, fail);
-    }
-  }
-
-  __device__ __forceinline__ void run() {
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_full);
-    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
-    const int NS = G.nstage;
-    int cur_u = -1;
-    UnitView uv;
-    ChunkIter ci(P, G);
-    for (; ci.valid(); ci.next()) {
-      const unsigned it = ci.it;
-      const int slot_i = (int)(it % NS);
-      // A failed wait sets the CTA's abort flag; this warp then runs on in skip mode (reads of
-      // in-bounds shared memory only) and every collective wait below returns at once.
-      const bool fail = !wait_mbar(P, sm, &full[slot_i], (it / NS) & 1u, DE_TIMEOUT_FULL);
-      const ChunkView cv = ci.view(G);
-      if (cv.u != cur_u) {
-        cur_u = cv.u;
-        uv = unit_view(P, G, cv.u);
-      }
-      const uint8_t* slot = smem + G.o_ring + (size_t)slot_i * G.stage_bytes;
-      bool ok;
-      if (cv.phase == P_ROUTER || cv.phase == P_SGU || cv.phase == P_RGU) ok = ensure_x(cv.u, uv);
-      else if (cv.phase == P_SDN) ok = ensure_xs(cv.u, uv);
-      else ok = ensure_xd(cv.u, uv);
-      if (!ok) break;
-      if (cv.c == 0 && uv.h_trace && !fail)
-        for (int c = ctid(); c < G.H; c += kConsumers) uv.h_trace[c] = __ldcg(uv.xin + c);
-      float* part = boxes + (size_t)(it % kBoxes) * G.box_floats;
-      if (cv.phase == P_ROUTER)
-        router_chunk(cv, slot, &empty[slot_i], part, it);
-      else if (G.bits == 4)
-        dispatch<4>(cv, uv, slot, &empty[slot_i], part, it, fail);
-      else
-        dispatch<2>(cv, uv, slot, &empty[slot_i], part, it, fail);
-      // this warp's share of the chunk's slot is written: tell the signal warp
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) red_release_cta_smem(&sm->done_count, 1u);
-    }
-    consumer_sync();  // every consumer warp's last delivery is published before this
-    if (ctid() == 0) sm->cons_done = 1;
-    // drain: never leave the CTA with bulk copies in flight
-    if (ctid() == 0 && sm->abort) {
-      const uint64_t deadline = global_ns() + 100000000ull;
-      while (!sm->prod_done && global_ns() < deadline) __nanosleep(1000);
-      const unsigned issued = sm->issued;
-      for (unsigned j = ci.it; j < issued; ++j) {
-        const int si = (int)(j % NS);
-        while (!mbar_try_wait(&full[si], (j / NS) & 1u) && global_ns() < deadline) {
-        }
-      }
-    }
-  }
-};
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     engine_kernel(const __grid_constant__ Prog P, const __grid_constant__ Geo G) {
@@ -1096,29 +1009,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
   if (threadIdx.x == 0) {
     sm->abort = 0;
-    sm->prod_done = 0;
+    sm->x_ready = 0;
+    sm->rt_ready = 0;
+    sm->xd_ready = 0;
+    for (int c = 0; c < CL_COUNT; ++c) sm->run_cnt[c] = 0;
     sm->issued = 0;
-    sm->done_count = 0;
-    sm->sig_done = 0;
-    sm->cons_done = 0;
     for (int i = 0; i < G.nstage; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kConsumerWarps);
+      mbar_init(&empty[i], 1);
     }
+    mbar_init(&sm->xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   if (warp == 0) {
-    producer(P, G, smem, sm);
+    if ((threadIdx.x & 31) == 0) producer(P, G, smem, sm);
     return;
   }
   if (warp == 1) {
-    signaller(P, G, smem, sm);
+    stager(P, G, smem, sm);
     return;
   }
-  Consumer c(P, G, smem, sm);
-  c.run();
+  consumer(P, G, smem, sm, warp - kCtrlWarps);
 }
 
 }  // namespace fmoe

@@ -1,40 +1,45 @@
 // engine.h — host/device description of one launch of the MoE engine kernel.
 //
 // A launch runs a sequence of "units"; a unit is one MoE layer applied to one token. The work
-// of a unit is cut into chunks, listed in dependency order by phase:
-//   P_ROUTER   router rows (fp32, binary64 accumulation) + the shared-gate row; the CTA whose
-//              completion brings the router count to its target selects the top-K experts
-//   P_SGU      shared expert gate/up rows + SwiGLU            (needs x)
-//   P_SDN      shared expert down rows + residual             (needs the shared h and sigma)
-//   P_RGU      routed experts gate/up rows + SwiGLU           (needs the routing decision)
-//   P_RDN      routed experts down rows + weighted combine    (needs all routed h)
-// Chunk g of the launch (g = unit * chunks_per_unit + index) belongs to CTA g mod gridDim, and
-// every CTA works through its chunks in increasing g; every wait a chunk makes is on chunks with
-// smaller g, so with all CTAs resident (one per SM) the schedule cannot deadlock, and every wait
-// is bounded in time in any case.
+// of a unit is cut into chunks of one shared-memory stage each, listed in dependency order:
+//   K_ROUTER  a column segment of one or more router rows (fp32 weights, binary64 sums); the
+//             shared-gate vector is router row E
+//   K_SGU     R rows of the shared expert's gate matrix and the same R rows of its up matrix
+//   K_RGU     the same for routed expert k (needs the routing decision)
+//   K_DN      Rd output rows of the fused down projection: output row j is the dot product of
+//             the concatenated rows j of every active down matrix (shared expert first, then
+//             routed k = 0..K-1) with the concatenated inputs [sigma*h_s | w_0*h_0 | ...]
+// Completion is counted per class: CL_ROUTER (router chunks), CL_GU (shared and routed gate/
+// up chunks) and CL_DN. Chunk g of the launch (g = unit * chunks_per_unit + index) belongs to
+// CTA g mod gridDim; inside a CTA, local chunk i goes to consumer warp i mod kConsumerWarps and
+// ring stage i mod nstage. Every wait a chunk makes is on chunks with smaller g, so with all
+// CTAs resident (one per SM) the schedule cannot deadlock, and every wait is bounded in time.
 #pragma once
 #include <stdint.h>
 
 namespace fmoe {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;    // 256 consumer threads
-constexpr int kThreads = kConsumers + 64;          // + one producer warp + one signal warp
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kCtrlWarps = 2;                      // producer + stager
+constexpr int kThreads = kConsumers + 32 * kCtrlWarps;
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
-constexpr int kMaxSlices = 256;                    // 32-column slices per (virtual) row
-constexpr int kSliceCols = 32;
-constexpr int kBoxes = 4;                          // outbox depth (chunks)
+constexpr int kRowsPerLane = 8;                    // rows one lane accumulates per chunk
+constexpr int kStageTarget = 9216;                 // bytes of weights per chunk (target)
+constexpr int kMaxStages = 32;
 
-enum Phase { P_ROUTER = 0, P_SGU = 1, P_SDN = 2, P_RGU = 3, P_RDN = 4, P_COUNT = 5 };
+enum Kind { K_ROUTER = 0, K_SGU = 1, K_RGU = 2, K_DN = 3, K_COUNT = 4 };
+enum Class { CL_ROUTER = 0, CL_GU = 1, CL_DN = 2, CL_COUNT = 3 };
 
-// Control words (uint32, zeroed before every launch). Phase counters take one atomic per CTA
-// per run of chunks; the CTA whose atomic completes a phase of a unit writes "phase p of unit
-// u is complete" into every CTA's own flag line, and waiters poll only their own line.
+// Control words (uint32, zeroed before every launch). Class counters take one atomic per CTA
+// per run of same-class chunks; the CTA whose atomic completes a class for a unit writes
+// "class c of unit u is complete" into every CTA's own flag line, and waiters poll only their
+// own line.
 enum Ctrl {
-  C_CNT = 0,                    // C_CNT + 32*phase: chunks of that phase completed (all units)
-  C_WORDS = 32 * P_COUNT,       // every counter on its own 128-byte line
-  F_WORDS = 32                  // per-CTA flag line: word p = units whose phase p is complete
+  C_CNT = 0,                    // C_CNT + 32*class: chunks of that class completed (all units)
+  C_WORDS = 32 * CL_COUNT,      // every counter on its own 128-byte line
+  F_WORDS = 32                  // per-CTA flag line: word c = units whose class c is complete
 };
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
@@ -47,39 +52,47 @@ struct LayerW {
   const float* gate;           // nullable [H]
 };
 
+// Lane layout of a dot-product chunk inside one warp: S lanes share a row (S a power of two,
+// >= the row's 32-column slices when they are fewer than 32), P = 32 / S rows side by side.
+struct LaneMap {
+  int nsl;                     // 32-column slices per (virtual) row
+  int S, P;                    // lanes per row, rows side by side
+  int nrl;                     // rows per lane (<= kRowsPerLane)
+};
+
 struct Geo {
   int H, I, E, K, bits;
   int route_on, shared_on, routed_on, gate_on;
-  // bytes per row
-  unsigned rc_h, rs_h, rc_i, rs_i;
-  unsigned long long q_gu, q_dn;  // bytes of an I x H (gate/up) and an H x I (down) packed matrix
-  // rows per chunk
-  int rr, rcg, rsd, rrd;
+  unsigned rc_h, rs_h, rc_i, rs_i;  // bytes per row of codes / scale-bias words (H or I wide)
+  unsigned long long q_gu;          // bytes of one I x H packed matrix (gate or up)
+  // router chunks
   int nr;                      // router rows: E + gate_on
-  int nb;                      // gate/up chunks per expert
-  int n[P_COUNT];
-  int off[P_COUNT + 1];        // off[P_COUNT] = chunks per unit
-  // thread mapping: slices of 32 columns, padded per virtual row
-  int sl_h, sp_h, p_h;         // H-wide rows (gate/up)
-  int sl_i, sp_i, p_i;         // I-wide rows (shared down)
-  int sl_d, sp_d, p_d;         // K*I-wide virtual rows (routed down)
-  int w_gu, w_sd, w_rd;        // waves per chunk
+  int rseg;                    // column segments per router row
+  int rcols;                   // columns per segment (H / rseg)
+  int rrows;                   // router rows per chunk (1 when rseg > 1)
+  int nrb;                     // router row blocks: ceil(nr / rrows)
+  // gate/up chunks
+  int R;                       // rows of gate (and as many of up) per chunk
+  int nb;                      // chunks per expert: ceil(I / R)
+  // down chunks
+  int nseg;                    // segments of a down virtual row: shared_on + K (routed)
+  int Rd;                      // virtual rows per chunk
+  int n[K_COUNT];
+  int off[K_COUNT + 1];        // off[K_COUNT] = chunks per unit
+  int ncl[CL_COUNT];           // chunks per unit of each class
+  LaneMap gu, dn;
   // shared memory carve-up (byte offsets from the dynamic smem base)
   unsigned stage_bytes;
   int nstage;
-  unsigned o_ring, o_full, o_empty, o_meta, o_xr, o_xg, o_sxg, o_xs, o_sxs, o_xd, o_sxd, o_red,
-      o_rows, o_misc;
+  unsigned o_ring, o_full, o_empty, o_xa, o_sxa, o_xg, o_sxg, o_red, o_misc;
   unsigned smem_bytes;
-  unsigned o_box;              // reduction slots: kBoxes x box_floats (partials + prefetched base)
-  int box_floats;
-  int red_part;                // floats of per-warp partials at the start of a slot (then bases)
 };
 
 struct Scratch {
   unsigned* ctrl;        // C_WORDS
   unsigned* flags;       // [gridDim][F_WORDS]
   int* err;              // sticky per-device error word
-  double* logits;        // [2][nr]
+  double* logits;        // [2][rseg][nr] partial logits per column segment
   float* hs;             // [2][I]
   float* hk;             // [2][K][I]
   float* normsq;         // [n_units]

@@ -1,5 +1,5 @@
 // ptx.cuh — thin inline-PTX wrappers for sm_100a: mbarriers, 1-D TMA bulk copies (no
-// multicast), acquire/release global accesses, the global timer and named barriers.
+// multicast), acquire/release accesses and atomics, proxy fences and the global timer.
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -101,24 +101,30 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
   return old;
 }
 
-// Barrier among the consumer warps only (id 1); the producer and signal warps never join it.
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
+__device__ __forceinline__ unsigned atom_add_acq_rel_cta_smem(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old)
+               : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return old;
 }
 
-// Barrier among the consumer warps that also ORs a predicate: every participant gets the same
-// answer, so a decision taken on it (abort or continue) is uniform across the consumers.
-__device__ __forceinline__ bool consumer_any(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v)
-      : "memory");
-  return r != 0;
+__device__ __forceinline__ unsigned atom_exch_cta_smem(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.relaxed.cta.shared::cta.exch.b32 %0, [%1], %2;" : "=r"(old)
+               : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void st_release_cta_smem(unsigned* p, unsigned v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Orders this thread's earlier generic-proxy accesses before its later async-proxy (bulk
+// copy) accesses, in every state space.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async;" ::: "memory");
 }
 
 __device__ __forceinline__ float4 ldcg4(const float* p) {
