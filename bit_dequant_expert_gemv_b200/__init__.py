@@ -38,6 +38,7 @@ _SIGS = {
     "fmoe_expert_gemv": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                                    C.c_void_p, C.c_void_p]),
     "fmoe_moe_layer": (C.c_int, [C.c_void_p] * 8),
+    "fmoe_moe_layer_noalloc": (C.c_int, [C.c_void_p] * 8),
     "fmoe_moe_layer_seq": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "fmoe_moe_layer_seq_host": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int,
@@ -193,6 +194,22 @@ def moe_layer(desc: LayerDesc, x, residual=None, bias=None, out=None, idx=None, 
     _ck("fmoe_moe_layer", lib().fmoe_moe_layer(arr, _ptr(x), _ptr(residual), _ptr(bias), _ptr(out),
                                               _ptr(idx), _ptr(weight), _stream(stream)))
     return out
+
+
+def moe_layer_noalloc(desc: LayerDesc, x, residual=None, bias=None, out=None, idx=None,
+                      weight=None, stream=None):
+    """fmoe_moe_layer_noalloc: one token with the library's fixed scratch array (no device
+    allocation inside the call; `out` must be given by callers that allocate nothing)."""
+    import torch
+    out = torch.empty_like(x) if out is None else out
+    arr, _ = _descs(desc)
+    _ck("fmoe_moe_layer_noalloc",
+        lib().fmoe_moe_layer_noalloc(arr, _ptr(x), _ptr(residual), _ptr(bias), _ptr(out),
+                                     _ptr(idx), _ptr(weight), _stream(stream)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 128 * 1024
 
 
 def moe_layer_seq(descs, x, residual=None, bias=None, out=None, idx=None, weight=None,

@@ -62,6 +62,16 @@ struct DevState {
 std::mutex g_mu;
 DevState g_dev[64];
 
+// State of fmoe_moe_layer_noalloc, set up on its first call on a device. `base` is the device
+// address of the fixed scratch array; its last 256 bytes hold the sticky error word.
+struct NoAllocState {
+  bool init = false;
+  int sms = 0;
+  int max_smem = 0;
+  uint8_t* base = nullptr;
+};
+NoAllocState g_na[64];
+constexpr size_t kNoAllocErrOff = FMOE_NOALLOC_SCRATCH_BYTES - 256;
 
 int dev_state(DevState** out) {
   int dev = 0;
@@ -361,8 +371,19 @@ int fmoe_sync_status(void* stream) {
   CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   int v = 0;
   CK(cudaMemcpy(&v, d->err, sizeof v, cudaMemcpyDeviceToHost));
+  if (v != 0) CK(cudaMemset(d->err, 0, sizeof(int)));
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (g_na[dev].init) {  // the fixed-scratch entry point keeps its own error word
+    int* na_err = reinterpret_cast<int*>(g_na[dev].base + kNoAllocErrOff);
+    int w = 0;
+    CK(cudaMemcpy(&w, na_err, sizeof w, cudaMemcpyDeviceToHost));
+    if (w != 0) {
+      CK(cudaMemset(na_err, 0, sizeof(int)));
+      if (v == 0) v = w;
+    }
+  }
   if (v == 0) return FMOE_OK;
-  CK(cudaMemset(d->err, 0, sizeof(int)));
   static const char* what[] = {"", "waiting for a weight stage", "waiting for a free stage",
                                "waiting for the routing decision", "waiting for a dependency",
                                "draining copies"};
@@ -540,6 +561,61 @@ int fmoe_moe_layer(const fmoe_layer_desc* layer, const float* x, const float* re
                    const float* logit_bias, float* out, int32_t* idx_out, float* w_out,
                    void* stream) {
   return fmoe_moe_layer_seq(layer, 1, x, residual, 1, logit_bias, out, idx_out, w_out, stream);
+}
+
+// ---------------------------------------------------------------- fixed-scratch variant
+// The scratch of fmoe_moe_layer_noalloc: one array per device, reserved with the library's
+// module image when it is loaded, so that the call itself never allocates.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FMOE_NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_state(NoAllocState** out) {
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FMOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  NoAllocState& s = g_na[dev];
+  if (!s.init) {
+    CK(cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev));
+    CK(cudaDeviceGetAttribute(&s.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    void* p = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    CK(cudaMemset(static_cast<uint8_t*>(p) + kNoAllocErrOff, 0, sizeof(int)));
+    CK(fmoe_engine_configure(s.max_smem));
+    s.base = static_cast<uint8_t*>(p);
+    s.init = true;
+  }
+  *out = &s;
+  return FMOE_OK;
+}
+
+int fmoe_moe_layer_noalloc(const fmoe_layer_desc* layer, const float* x, const float* residual,
+                           const float* logit_bias, float* out, int32_t* idx_out, float* w_out,
+                           void* stream) {
+  NoAllocState* s;
+  int rc = noalloc_state(&s);
+  if (rc) return rc;
+  DevState shape_limits;  // prep_layers only reads the shared-memory limit
+  shape_limits.sms = s->sms;
+  shape_limits.max_smem = s->max_smem;
+  Geo G;
+  if ((rc = prep_layers(layer, 1, &shape_limits, &G))) return rc;
+  if (!x || !out) return fail(FMOE_ERR_INVALID, "x and out are required");
+  if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
+    return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
+  if (x == out) return fail(FMOE_ERR_INVALID, "x must not alias out");
+  const ScratchPlan sp = plan_scratch(G, 1, s->sms);
+  if (sp.total > kNoAllocErrOff)
+    return fail(FMOE_ERR_UNSUPPORTED,
+                "fmoe_moe_layer_noalloc: this shape needs %zu bytes of scratch, the fixed area "
+                "holds %zu",
+                sp.total, kNoAllocErrOff);
+  Prog P;
+  base_prog(&P, MODE_SEQ);
+  P.n_units = 1; P.n_layers = 1; P.n_tokens = 1;
+  P.x = x; P.res = residual; P.out = out; P.bias = logit_bias; P.idx_out = idx_out; P.w_out = w_out;
+  fill_layers(&P, layer, 1);
+  bind_scratch(&P, sp, s->base, reinterpret_cast<int*>(s->base + kNoAllocErrOff));
+  return enqueue_engine(&P, G, sp, s->base, s->sms, static_cast<cudaStream_t>(stream));
 }
 
 static int stack_prog(const fmoe_layer_desc* layers, int n_layers, const float* h_in,
