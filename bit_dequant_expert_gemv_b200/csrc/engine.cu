@@ -175,10 +175,14 @@ __device__ __forceinline__ unsigned local_chunks(const Prog& P, const Geo& G) {
 // ------------------------------------------------------------------------------------------
 struct Smem {  // small shared state (in the misc area)
   uint64_t xbar;               // the stager's TMA barrier
+  // Readiness per unit: a monotone counter (units ready so far; the truth) and an mbarrier
+  // that completes one phase per unit, used only to sleep until the next increment. Waiters
+  // may run several units ahead of the stager, so the counter decides, never the parity.
+  uint64_t x_bar;              // x staged
+  uint64_t rt_bar;             // routing decision in rt_e / rt_w
+  uint64_t xd_bar;             // down input staged
+  unsigned x_ready, rt_ready, xd_ready;
   volatile int abort;
-  unsigned x_ready;            // units whose x is staged          (release/acquire, CTA)
-  unsigned rt_ready;           // units whose routing is in rt_*   (release/acquire, CTA)
-  unsigned xd_ready;           // units whose down input is staged (release/acquire, CTA)
   unsigned run_cnt[CL_COUNT];  // chunks of the current run of each class finished here
   volatile unsigned issued;    // chunks the producer has issued
   int rt_e[2][kMaxK];          // routing of unit u (index u & 1): experts and weights
@@ -213,34 +217,44 @@ __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a
   }
 }
 
-// Same on a CTA-local counter in shared memory.
-__device__ __noinline__ bool spin_geq_smem(const Prog& P, Smem* sm, const unsigned* a,
-                                           unsigned target, int code) {
-  if ((int)(ld_acquire_cta_smem(a) - target) >= 0) return true;
-  const uint64_t deadline = global_ns() + P.wait_ns;
-  for (unsigned it = 0;; ++it) {
-    if ((int)(ld_acquire_cta_smem(a) - target) >= 0) return true;
-    if (sm->abort) return false;
-    if ((it & 63) == 63 && global_ns() > deadline) {
-      raise_error(P, sm, code);
-      return false;
-    }
-    __nanosleep(32);
-  }
-}
-
 __device__ __forceinline__ bool wait_mbar(const Prog& P, Smem* sm, uint64_t* bar, unsigned parity,
                                           int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
-  for (unsigned it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
     if (sm->abort) return false;
-    if ((it & 63) == 63 && global_ns() > deadline) {
+    if (global_ns() > deadline) {
       raise_error(P, sm, code);
       return false;
     }
   }
+}
+
+// Wait until the readiness counter *cnt reaches target. Sleeps on the phase that the next
+// increment completes (the stager stores the counter before it arrives on the barrier), and
+// re-reads the counter after every wake-up or after at most ~1 us.
+__device__ __noinline__ bool wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
+                                        uint64_t* bar, unsigned target, int code) {
+  unsigned c = ld_acquire_cta_smem(cnt);
+  if ((int)(c - target) >= 0) return true;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+  for (;;) {
+    mbar_try_wait_sleep(bar, c & 1u, 1000u);
+    c = ld_acquire_cta_smem(cnt);
+    if ((int)(c - target) >= 0) return true;
+    if (sm->abort) return false;
+    if (global_ns() > deadline) {
+      raise_error(P, sm, code);
+      return false;
+    }
+  }
+}
+
+// the stager's side: publish "unit u is ready" on a counter and wake sleepers
+__device__ __forceinline__ void signal_ready(unsigned* cnt, uint64_t* bar, int u) {
+  st_release_cta_smem(cnt, (unsigned)(u + 1));
+  mbar_arrive(bar);
 }
 
 // Whole-warp wrappers: lane 0 waits, every lane gets the verdict, and what was published
@@ -254,10 +268,10 @@ __device__ __forceinline__ bool warp_wait_flag(const Prog& P, Smem* sm, int cls,
   return ok != 0;
 }
 
-__device__ __forceinline__ bool warp_wait_smem(const Prog& P, Smem* sm, const unsigned* a,
-                                               unsigned target, int code) {
+__device__ __forceinline__ bool warp_wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
+                                                uint64_t* bar, unsigned target, int code) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = spin_geq_smem(P, sm, a, target, code);
+  if ((threadIdx.x & 31) == 0) ok = wait_ready(P, sm, cnt, bar, target, code);
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;
@@ -328,7 +342,8 @@ __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
         chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
     const bool routed = cv.kind == K_RGU || (cv.kind == K_DN && G.routed_on);
     if (routed && cv.u != rt_u) {
-      if (!spin_geq_smem(P, sm, &sm->rt_ready, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE)) break;
+      if (!wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE))
+        break;
       for (int k = 0; k < G.K; ++k) eidx[k] = min(max(sm->rt_e[cv.u & 1][k], 0), G.E - 1);
       rt_u = cv.u;
     }
@@ -476,13 +491,26 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
 #pragma unroll
   for (int i = 0; i < kPer; ++i) best[i] = 0ull;
   for (int e0 = 0; e0 < G.E; e0 += 32 * kPer) {
+    // all loads of a segment are independent, so each segment costs one round trip
+    double lv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ec = min(e0 + lane + 32 * i, G.E - 1);
+      lv[i] = bias ? (double)__ldcg(bias + ec) : 0.0;
+    }
+    for (int s = 0; s < G.rseg; ++s) {
+      double part[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        part[i] = __ldcg(lg + (size_t)s * G.nr + min(e0 + lane + 32 * i, G.E - 1));
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) lv[i] += part[i];
+    }
     unsigned long long key[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int e = e0 + lane + 32 * i;
-      const int ec = min(e, G.E - 1);
-      const double l = unit_logit(G, lg, ec) + (bias ? (double)__ldcg(bias + ec) : 0.0);
-      key[i] = e < G.E ? pkey(l, e) : 0ull;
+      key[i] = e < G.E ? pkey(lv[i], e) : 0ull;
     }
     sort16_desc(key);
     if (e0 == 0) {
@@ -549,14 +577,17 @@ __device__ __forceinline__ float4 xform(float4 v, int bits) {
                      v.w * 0.015625f - v.z * 0.0625f);
 }
 
-// Bring `bytes` from global memory (written by other CTAs or by the caller) into shared
-// memory with one bulk copy and wait for it.
+// Bring up to two blocks from global memory (written by other CTAs or by the caller) into
+// shared memory with bulk copies on one barrier, and wait for both.
 __device__ __forceinline__ bool stage_in(const Prog& P, Smem* sm, void* dst, const void* src,
-                                         unsigned bytes, unsigned& xphase) {
+                                         unsigned bytes, unsigned& xphase,
+                                         void* dst2 = nullptr, const void* src2 = nullptr,
+                                         unsigned bytes2 = 0) {
   if ((threadIdx.x & 31) == 0) {
-    fence_proxy_async();  // order earlier generic accesses before the async-proxy copy
-    mbar_arrive_expect_tx(&sm->xbar, bytes);
-    tma_load_1d(dst, src, bytes, &sm->xbar);
+    fence_proxy_async();  // order earlier generic accesses before the async-proxy copies
+    mbar_arrive_expect_tx(&sm->xbar, bytes + bytes2);
+    if (bytes) tma_load_1d(dst, src, bytes, &sm->xbar);
+    if (bytes2) tma_load_1d(dst2, src2, bytes2, &sm->xbar);
   }
   const bool ok = warp_wait_mbar(P, sm, &sm->xbar, xphase, DE_TIMEOUT_DEP);
   xphase ^= 1u;
@@ -616,6 +647,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     if (owner && uv.h_trace)
       for (int c = lane * 4; c < G.H; c += 128)
         *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XA + c);
+    __syncwarp();  // every lane has read the raw x before any lane rescales it in place
     if (gu_on) {
       transform_slices(XA, XG, SXG, G.H / 32, G.bits, [&](int) { return f; },
                        G.route_on && uv.norm);
@@ -627,7 +659,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       }
     }
     __syncwarp();
-    if (lane == 0) st_release_cta_smem(&sm->x_ready, (unsigned)(u + 1));
+    if (lane == 0) signal_ready(&sm->x_ready, &sm->x_bar, u);
     // ---- routing decision: needs every router chunk of unit u
     float sigma = 1.f;
     if (G.route_on) {
@@ -638,18 +670,16 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
                 owner ? uv.w_out : nullptr);
       __syncwarp();
-      if (lane == 0) st_release_cta_smem(&sm->rt_ready, (unsigned)(u + 1));
+      if (lane == 0) signal_ready(&sm->rt_ready, &sm->rt_bar, u);
     }
     // ---- down input [sigma*h_s | w_0*h_0 | ...]: needs every gate/up chunk of unit u
     if (G.nseg > 0) {
       if (!warp_wait_flag(P, sm, CL_GU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
-      bool ok = true;
-      if (G.shared_on)
-        ok = stage_in(P, sm, XA, P.s.hs + (size_t)uv.slot * G.I, 4u * (unsigned)G.I, xphase);
-      if (ok && G.routed_on)
-        ok = stage_in(P, sm, XA + (size_t)G.shared_on * G.I,
-                      P.s.hk + (size_t)uv.slot * G.K * G.I, 4u * (unsigned)(G.K * G.I), xphase);
-      if (!ok) break;
+      const unsigned bs = G.shared_on ? 4u * (unsigned)G.I : 0u;
+      const unsigned bk = G.routed_on ? 4u * (unsigned)(G.K * G.I) : 0u;
+      if (!stage_in(P, sm, XA, P.s.hs + (size_t)uv.slot * G.I, bs, xphase,
+                    XA + (size_t)G.shared_on * G.I, P.s.hk + (size_t)uv.slot * G.K * G.I, bk))
+        break;
       const int spseg = G.I / 32;
       const float* rw = sm->rt_w[u & 1];
       transform_slices(
@@ -660,7 +690,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
           },
           false);
       __syncwarp();
-      if (lane == 0) st_release_cta_smem(&sm->xd_ready, (unsigned)(u + 1));
+      if (lane == 0) signal_ready(&sm->xd_ready, &sm->xd_bar, u);
     }
   }
 }
@@ -988,8 +1018,10 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
       cur_u = cv.u;
       uv = unit_view(P, G, cv.u);
     }
-    const unsigned* ready = cv.kind == K_DN ? &sm->xd_ready : &sm->x_ready;
-    if (!warp_wait_smem(P, sm, ready, (unsigned)(cv.u + 1), DE_TIMEOUT_DEP)) break;
+    const bool dn = cv.kind == K_DN;
+    if (!warp_wait_ready(P, sm, dn ? &sm->xd_ready : &sm->x_ready, dn ? &sm->xd_bar : &sm->x_bar,
+                         (unsigned)(cv.u + 1), DE_TIMEOUT_DEP))
+      break;
     const uint8_t* stage = smem + G.o_ring + (size_t)slot * G.stage_bytes;
     if (cv.kind == K_ROUTER)
       router_chunk(P, G, cv, stage, &empty[slot], XR);
@@ -1009,11 +1041,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
   if (threadIdx.x == 0) {
     sm->abort = 0;
-    sm->x_ready = 0;
-    sm->rt_ready = 0;
-    sm->xd_ready = 0;
     for (int c = 0; c < CL_COUNT; ++c) sm->run_cnt[c] = 0;
     sm->issued = 0;
+    sm->x_ready = sm->rt_ready = sm->xd_ready = 0;
+    mbar_init(&sm->x_bar, 1);
+    mbar_init(&sm->rt_bar, 1);
+    mbar_init(&sm->xd_bar, 1);
     for (int i = 0; i < G.nstage; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
