@@ -196,12 +196,17 @@ __device__ __forceinline__ void raise_error(const Prog& P, Smem* sm, int code) {
 
 // Spin until *a - target >= 0 (wrap-safe) on a gpu-scope flag, the budget runs out, the CTA
 // aborts or another CTA has recorded an error.
+// Polls with relaxed loads (an acquire per poll would be a gpu-scope ordering operation each
+// time) and makes one acquire fence once the flag is seen.
 __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a, unsigned target,
                                       int code) {
   if ((int)(ld_acquire(a) - target) >= 0) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
   for (unsigned it = 0;; ++it) {
-    if ((int)(ld_acquire(a) - target) >= 0) return true;
+    if ((int)(ld_relaxed_gpu(a) - target) >= 0) {
+      fence_acq_rel_gpu();
+      return true;
+    }
     if (sm->abort) return false;
     if ((it & 15) == 15) {
       if (ld_volatile_int(P.s.err) != 0) {
@@ -220,33 +225,39 @@ __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a
 __device__ __forceinline__ bool wait_mbar(const Prog& P, Smem* sm, uint64_t* bar, unsigned parity,
                                           int code) {
   if (mbar_try_wait(bar, parity)) return true;
+  // back off between polls: every poll is a shared-memory operation that competes with the
+  // working warps' loads
   const uint64_t deadline = global_ns() + P.wait_ns;
+  unsigned ns = 32;
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
     if (sm->abort) return false;
     if (global_ns() > deadline) {
       raise_error(P, sm, code);
       return false;
     }
+    ns = ns < 256 ? 2 * ns : 256;
   }
 }
 
 // Wait until the readiness counter *cnt reaches target. Sleeps on the phase that the next
 // increment completes (the stager stores the counter before it arrives on the barrier), and
 // re-reads the counter after every wake-up or after at most ~1 us.
-__device__ __noinline__ bool wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
-                                        uint64_t* bar, unsigned target, int code) {
+// Returns the counter value seen (>= target), or 0 if the wait failed.
+__device__ __noinline__ unsigned wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
+                                            uint64_t* bar, unsigned target, int code) {
   unsigned c = ld_acquire_cta_smem(cnt);
-  if ((int)(c - target) >= 0) return true;
+  if ((int)(c - target) >= 0) return c;
   const uint64_t deadline = global_ns() + P.wait_ns;
   for (;;) {
-    mbar_try_wait_sleep(bar, c & 1u, 1000u);
+    if (!mbar_try_wait_sleep(bar, c & 1u, 1000u)) __nanosleep(256);
     c = ld_acquire_cta_smem(cnt);
-    if ((int)(c - target) >= 0) return true;
-    if (sm->abort) return false;
+    if ((int)(c - target) >= 0) return c;
+    if (sm->abort) return 0u;
     if (global_ns() > deadline) {
       raise_error(P, sm, code);
-      return false;
+      return 0u;
     }
   }
 }
@@ -268,13 +279,14 @@ __device__ __forceinline__ bool warp_wait_flag(const Prog& P, Smem* sm, int cls,
   return ok != 0;
 }
 
-__device__ __forceinline__ bool warp_wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
-                                                uint64_t* bar, unsigned target, int code) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = wait_ready(P, sm, cnt, bar, target, code);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
+// Returns the number of ready units seen (>= target), or 0 if the wait failed.
+__device__ __forceinline__ unsigned warp_wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
+                                                    uint64_t* bar, unsigned target, int code) {
+  unsigned c = 0;
+  if ((threadIdx.x & 31) == 0) c = wait_ready(P, sm, cnt, bar, target, code);
+  c = __shfl_sync(0xffffffffu, c, 0);
   __syncwarp();
-  return ok != 0;
+  return c;
 }
 
 __device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t* bar,
@@ -289,20 +301,21 @@ __device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t
 // ------------------------------------------------------------------------------------------
 // completion of a chunk: counted per run of same-class chunks, published per run
 // ------------------------------------------------------------------------------------------
-// Called by the whole warp after every global store of the chunk was issued. The warp whose
-// chunk completes its CTA's run of (unit, class) orders the run's stores of every warp of the
-// CTA (CTA-scope acquire of the run counter, then a gpu-scope fence) before its atomic on the
-// class counter; the warp whose atomic completes the class for the unit writes the flag of
-// every CTA (release stores).
-__device__ __forceinline__ void finish_chunk(const Prog& P, const Geo& G, Smem* sm, int cls,
-                                             int u) {
+// Called by the whole warp after the global stores of its last chunk of a run were issued,
+// with `mine` = the number of chunks of the run this warp did. One CTA-scope release-acquire
+// add per warp and run; the warp that completes the CTA's run of (unit, class) orders every
+// warp's stores of the run (CTA-scope acquire, then a gpu-scope fence) before its atomic on
+// the class counter, and the warp whose atomic completes the class for the unit writes the
+// flag of every CTA (release stores).
+__device__ __forceinline__ void finish_run(const Prog& P, const Geo& G, Smem* sm, int cls, int u,
+                                           unsigned mine) {
   const int lane = threadIdx.x & 31;
   __syncwarp();
   int bcast = 0;
   if (lane == 0) {
-    const unsigned old = atom_add_acq_rel_cta_smem(&sm->run_cnt[cls], 1u);
+    const unsigned old = atom_add_acq_rel_cta_smem(&sm->run_cnt[cls], mine);
     const unsigned nrun = run_len(G, u, cls);
-    if (old + 1u == nrun) {
+    if (old + mine == nrun) {
       atom_exch_cta_smem(&sm->run_cnt[cls], 0u);
       fence_acq_rel_gpu();
       const unsigned og = atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cls), nrun);
@@ -311,9 +324,13 @@ __device__ __forceinline__ void finish_chunk(const Prog& P, const Geo& G, Smem* 
   }
   bcast = __shfl_sync(0xffffffffu, bcast, 0);
   if (bcast && !(cls == CL_ROUTER && (P.debug & 1))) {
+    // One fence per lane (after lane 0's acquire of the counter, through the warp sync), then
+    // relaxed stores: a release store each would wait for the previous one, and the CTAs
+    // served last would see the flag microseconds later.
     __syncwarp();
+    fence_acq_rel_gpu();
     for (int c = lane; c < (int)gridDim.x; c += 32)
-      st_release(P.s.flags + c * F_WORDS + cls, (unsigned)(u + 1));
+      st_relaxed_gpu(P.s.flags + c * F_WORDS + cls, (unsigned)(u + 1));
   }
 }
 
@@ -342,7 +359,7 @@ __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
         chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
     const bool routed = cv.kind == K_RGU || (cv.kind == K_DN && G.routed_on);
     if (routed && cv.u != rt_u) {
-      if (!wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE))
+      if (wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE) == 0u)
         break;
       for (int k = 0; k < G.K; ++k) eidx[k] = min(max(sm->rt_e[cv.u & 1][k], 0), G.E - 1);
       rt_u = cv.u;
@@ -706,9 +723,9 @@ __device__ __forceinline__ uint32_t magic_byte(uint32_t word, int k) {
 
 // acc[w] += s_w * sum(q x) + z_w * sum(x) over the slice, for W rows whose codes start at
 // stage + coff[w] and whose scale/bias word is at stage + soff[w]; rows with ok[w] false add
-// 0 (their offsets must still point inside the stage).
+// 0 (their offsets must still point inside the stage). xq: the slice's transformed x.
 template <int BITS, int W>
-__device__ __forceinline__ void qslice(const uint8_t* stage, const unsigned (&coff)[W],
+__device__ __forceinline__ void qslice(uint32_t stage, const unsigned (&coff)[W],
                                        const unsigned (&soff)[W], const bool (&ok)[W],
                                        const float (&xq)[32], float sx, float* acc) {
   constexpr int kWords = BITS == 4 ? 4 : 2;
@@ -717,13 +734,13 @@ __device__ __forceinline__ void qslice(const uint8_t* stage, const unsigned (&co
 #pragma unroll
   for (int w = 0; w < W; ++w) {
     if constexpr (BITS == 4) {
-      const uint4 t = *reinterpret_cast<const uint4*>(stage + coff[w]);
+      const uint4 t = lds128(stage + coff[w]);
       q[w][0] = t.x; q[w][1] = t.y; q[w][2] = t.z; q[w][3] = t.w;
     } else {
-      const uint2 t = *reinterpret_cast<const uint2*>(stage + coff[w]);
+      const uint2 t = lds64(stage + coff[w]);
       q[w][0] = t.x; q[w][1] = t.y;
     }
-    sbw[w] = *reinterpret_cast<const uint32_t*>(stage + soff[w]);
+    sbw[w] = lds32(stage + soff[w]);
   }
   const float2 m = make_float2(-32768.f, -32768.f);
   float2 a0[W], a1[W];
@@ -820,12 +837,13 @@ struct RowGeom {
 };
 
 // A chunk's rows x slices on one warp: rows rho = lane_p + P*i (i < NRL), slices
-// t = lane_s + S*j; rows are processed in lock-step groups of GW (3 or 4) per slice. The
-// reduced value of row rho ends in red[(rho % P) * kRowsPerLane + rho / P].
+// t = lane_s + S*j; rows are processed in lock-step groups of GW (3 or 4) per slice. Row rho
+// takes part when valid(rho). The reduced value of row rho ends in
+// red[(rho % P) * kRowsPerLane + rho / P].
 template <int BITS, int NRL, typename Valid>
-__device__ __forceinline__ void dot_chunk(const uint8_t* stage, const LaneMap& M,
-                                          const RowGeom& RG, int nrows, Valid valid,
-                                          const float* X, const float* SX, float* red) {
+__device__ __forceinline__ void dot_chunk(uint32_t st, const LaneMap& M, const RowGeom& RG,
+                                          int nrows, Valid valid, uint32_t xs, uint32_t sxs,
+                                          float* red) {
   constexpr int NRLP = NRL <= 4 ? 4 : 8;         // padded to a power of two for the butterfly
   constexpr int GW = (NRL % 4 == 0) ? 4 : 3;     // rows per lock-step group
   const int lane = threadIdx.x & 31;
@@ -842,10 +860,11 @@ __device__ __forceinline__ void dot_chunk(const uint8_t* stage, const LaneMap& M
     float xq[32];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 a = *reinterpret_cast<const float4*>(X + xpos(tc, i));
-      xq[4 * i] = a.x; xq[4 * i + 1] = a.y; xq[4 * i + 2] = a.z; xq[4 * i + 3] = a.w;
+      const uint4 a = lds128(xs + 4u * (unsigned)xpos(tc, i));
+      xq[4 * i] = __uint_as_float(a.x); xq[4 * i + 1] = __uint_as_float(a.y);
+      xq[4 * i + 2] = __uint_as_float(a.z); xq[4 * i + 3] = __uint_as_float(a.w);
     }
-    const float sx = SX[tc];
+    const float sx = __uint_as_float(lds32(sxs + 4u * (unsigned)tc));
     const int seg = tc / RG.spseg, loc = tc - seg * RG.spseg;
     const unsigned cbase = (unsigned)seg * RG.seg_c + (unsigned)loc * cb;
     const unsigned sbase = RG.sb0 + (unsigned)seg * RG.seg_s + (unsigned)(loc >> 1) * 4u;
@@ -862,7 +881,7 @@ __device__ __forceinline__ void dot_chunk(const uint8_t* stage, const LaneMap& M
           coff[w] = cbase + rr * RG.rc;
           soff[w] = sbase + rr * RG.rs;
         }
-        qslice<BITS, GW>(stage, coff, soff, ok, xq, sx, acc + g);
+        qslice<BITS, GW>(st, coff, soff, ok, xq, sx, acc + g);
       }
     }
   }
@@ -876,9 +895,11 @@ __device__ __forceinline__ float red_row(const float* red, const LaneMap& M, int
 // ------------------------------------------------------------------------------------------
 // consumer warps
 // ------------------------------------------------------------------------------------------
+// Every lane's reads of the stage have returned (their values fed the row sums already
+// reduced across the warp), so a relaxed arrival is enough to hand the stage back.
 __device__ __forceinline__ void release_stage(uint64_t* empty) {
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
+  if ((threadIdx.x & 31) == 0) mbar_arrive_relaxed(empty);
 }
 
 // router rows r0..r0+n-1, columns seg*rcols .. +rcols: binary64 sums of fp32 products
@@ -923,8 +944,9 @@ __device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, const Chun
   RG.spseg = G.H / 32;
   const int R = G.R, n = cv.n;
   dot_chunk<BITS, NRL>(
-      stage, G.gu, RG, 2 * R,
-      [&](int rho) { return rho < 2 * R && (rho < R ? rho : rho - R) < n; }, XG, SXG, red);
+      smem_u32(stage), G.gu, RG, 2 * R,
+      [&](int rho) { return rho < 2 * R && (rho < R ? rho : rho - R) < n; }, smem_u32(XG),
+      smem_u32(SXG), red);
   release_stage(empty);
   __syncwarp();
   float* h = cv.kind == K_SGU ? P.s.hs + (size_t)(cv.u & 1) * G.I
@@ -952,7 +974,8 @@ __device__ __forceinline__ void dn_chunk(const Prog& P, const Geo& G, const Chun
   RG.sb0 = (unsigned)G.nseg * G.Rd * G.rc_i;
   RG.spseg = G.I / 32;
   const int n = cv.n;
-  dot_chunk<BITS, NRL>(stage, G.dn, RG, n, [&](int rho) { return rho < n; }, XD, SXD, red);
+  dot_chunk<BITS, NRL>(smem_u32(stage), G.dn, RG, n, [&](int rho) { return rho < n; },
+                       smem_u32(XD), smem_u32(SXD), red);
   release_stage(empty);
   __syncwarp();
   float sq = 0.f;
@@ -1009,19 +1032,27 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
   const unsigned n_local = local_chunks(P, G);
   int cur_u = -1;
   UnitView uv;
+  unsigned x_seen = 0, xd_seen = 0;  // units known ready (counter values already acquired)
+  unsigned mine = 0;                 // chunks of the current run done by this warp
   for (unsigned i = (unsigned)w; i < n_local; i += kConsumerWarps) {
     const int slot = (int)(i % NS);
     if (!warp_wait_mbar(P, sm, &full[slot], (i / NS) & 1u, DE_TIMEOUT_FULL)) break;
-    const Chunk cv =
-        chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
+    const unsigned long long g = (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x;
+    const Chunk cv = chunk_at(G, g);
     if (cv.u != cur_u) {
       cur_u = cv.u;
       uv = unit_view(P, G, cv.u);
     }
-    const bool dn = cv.kind == K_DN;
-    if (!warp_wait_ready(P, sm, dn ? &sm->xd_ready : &sm->x_ready, dn ? &sm->xd_bar : &sm->x_bar,
-                         (unsigned)(cv.u + 1), DE_TIMEOUT_DEP))
-      break;
+    const unsigned need = (unsigned)(cv.u + 1);
+    if (cv.kind == K_DN) {
+      if ((int)(xd_seen - need) < 0) {
+        xd_seen = warp_wait_ready(P, sm, &sm->xd_ready, &sm->xd_bar, need, DE_TIMEOUT_DEP);
+        if (xd_seen == 0u) break;
+      }
+    } else if ((int)(x_seen - need) < 0) {
+      x_seen = warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, need, DE_TIMEOUT_DEP);
+      if (x_seen == 0u) break;
+    }
     const uint8_t* stage = smem + G.o_ring + (size_t)slot * G.stage_bytes;
     if (cv.kind == K_ROUTER)
       router_chunk(P, G, cv, stage, &empty[slot], XR);
@@ -1029,7 +1060,18 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
       dispatch_dot<4>(P, G, cv, uv, stage, &empty[slot], smem, red);
     else
       dispatch_dot<2>(P, G, cv, uv, stage, &empty[slot], smem, red);
-    finish_chunk(P, G, sm, class_of(cv.kind), cv.u);
+    ++mine;
+    // publish when this warp's next chunk belongs to another (unit, class) run, or there is none
+    const int cls = class_of(cv.kind);
+    bool run_end = i + kConsumerWarps >= n_local;
+    if (!run_end) {
+      const Chunk nx = chunk_at(G, g + (unsigned long long)kConsumerWarps * gridDim.x);
+      run_end = nx.u != cv.u || class_of(nx.kind) != cls;
+    }
+    if (run_end) {
+      finish_run(P, G, sm, cls, cv.u, mine);
+      mine = 0;
+    }
   }
 }
 

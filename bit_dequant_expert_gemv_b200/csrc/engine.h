@@ -26,7 +26,7 @@ constexpr int kThreads = kConsumers + 32 * kCtrlWarps;
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
 constexpr int kRowsPerLane = 8;                    // rows one lane accumulates per chunk
-constexpr int kStageTarget = 9216;                 // bytes of weights per chunk (target)
+constexpr int kStageTarget = 11520;                // bytes of weights per chunk (target)
 constexpr int kMaxStages = 32;
 
 enum Kind { K_ROUTER = 0, K_SGU = 1, K_RGU = 2, K_DN = 3, K_COUNT = 4 };
