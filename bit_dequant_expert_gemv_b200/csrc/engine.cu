@@ -99,15 +99,34 @@ struct Chunk {
   int u, c, kind, j, r0, n, k, seg;
 };
 
-__device__ __forceinline__ Chunk chunk_at(const Geo& G, unsigned long long g) {
-  const unsigned ntot = (unsigned)G.off[K_COUNT];
+// The chunks g0, g0 + step, g0 + 2 step, ... of a launch, walked without divisions: (u, c) is
+// the current chunk's unit and index within the unit (one division at the start only).
+struct ChunkWalk {
+  int u, c, step, ntot;
+  __device__ __forceinline__ void init(const Geo& G, unsigned long long g0, int step_) {
+    ntot = G.off[K_COUNT];
+    u = (int)(g0 / (unsigned)ntot);
+    c = (int)(g0 - (unsigned long long)u * (unsigned)ntot);
+    step = step_;
+  }
+  __device__ __forceinline__ void next() {
+    c += step;
+    while (c >= ntot) {
+      c -= ntot;
+      ++u;
+    }
+  }
+};
+
+// The chunk (u, c) decoded (no 64-bit arithmetic).
+__device__ __forceinline__ Chunk chunk_view(const Geo& G, int u, int c) {
   Chunk v;
-  v.u = (int)(g / ntot);
-  v.c = (int)(g - (unsigned long long)v.u * ntot);
+  v.u = u;
+  v.c = c;
   int kd = 0;
-  while (v.c >= G.off[kd + 1]) ++kd;
+  while (c >= G.off[kd + 1]) ++kd;
   v.kind = kd;
-  v.j = v.c - G.off[kd];
+  v.j = c - G.off[kd];
   v.k = 0;
   v.seg = 0;
   switch (kd) {
@@ -184,7 +203,6 @@ struct Smem {  // small shared state (in the misc area)
   unsigned x_ready, rt_ready, xd_ready;
   volatile int abort;
   unsigned run_cnt[CL_COUNT];  // chunks of the current run of each class finished here
-  volatile unsigned issued;    // chunks the producer has issued
   int rt_e[2][kMaxK];          // routing of unit u (index u & 1): experts and weights
   float rt_w[2][kMaxK];
 };
@@ -342,94 +360,174 @@ __device__ __forceinline__ void copy_rows(uint8_t* dst, const uint8_t* src, unsi
   if (bytes) tma_load_1d(dst, src, bytes, bar);
 }
 
+// One bulk copy of a chunk: copy number q of the chunk (q < copies_of(chunk)). Returns the
+// byte count (0 when chunk has no copy q) and sets the source and the offset in the stage.
+__device__ __forceinline__ unsigned copy_desc(const Geo& G, const LayerW& L, const Smem* sm,
+                                              const Chunk& cv, int q, const uint8_t** src,
+                                              unsigned* dst_off) {
+  switch (cv.kind) {
+    case K_ROUTER: {
+      if (G.rseg == 1) {  // whole rows r0 .. r0+n-1; row E is the shared-gate vector
+        const unsigned rowb = 4u * (unsigned)G.H;
+        const int a = cv.r0, b = min(cv.r0 + cv.n, G.E);
+        if (q == 0 && b > a) {
+          *src = reinterpret_cast<const uint8_t*>(L.router + (size_t)a * G.H);
+          *dst_off = 0;
+          return (unsigned)(b - a) * rowb;
+        }
+        if (q == 1 && cv.r0 + cv.n > G.E) {
+          *src = reinterpret_cast<const uint8_t*>(L.gate);
+          *dst_off = (unsigned)(G.E - cv.r0) * rowb;
+          return rowb;
+        }
+        return 0u;
+      }
+      if (q != 0) return 0u;  // one column segment of row r0
+      const float* row = cv.r0 < G.E ? L.router + (size_t)cv.r0 * G.H : L.gate;
+      *src = reinterpret_cast<const uint8_t*>(row + (size_t)cv.seg * G.rcols);
+      *dst_off = 0;
+      return 4u * (unsigned)G.rcols;
+    }
+    case K_SGU:
+    case K_RGU: {  // stage: gate codes | up codes | gate sb | up sb, R rows each
+      if (q >= 4) return 0u;
+      const uint8_t* base =
+          cv.kind == K_SGU
+              ? L.shared
+              : L.experts + (size_t)min(max(sm->rt_e[cv.u & 1][cv.k], 0), G.E - 1) * L.expert_stride;
+      const bool up = (q & 1) != 0, sbq = q >= 2;
+      const size_t mat = up ? G.q_gu : 0;
+      if (!sbq) {
+        *src = base + mat + (size_t)cv.r0 * G.rc_h;
+        *dst_off = (up ? (unsigned)G.R : 0u) * G.rc_h;
+        return (unsigned)cv.n * G.rc_h;
+      }
+      *src = base + mat + (size_t)G.I * G.rc_h + (size_t)cv.r0 * G.rs_h;
+      *dst_off = 2u * (unsigned)G.R * G.rc_h + (up ? (unsigned)G.R : 0u) * G.rs_h;
+      return (unsigned)cv.n * G.rs_h;
+    }
+    default: {  // K_DN: per segment s (shared first, then routed k) Rd rows of codes | sb
+      const int sgm = q >> 1;
+      if (sgm >= G.nseg) return 0u;
+      const uint8_t* eb =
+          (G.shared_on && sgm == 0)
+              ? L.shared
+              : L.experts + (size_t)min(max(sm->rt_e[cv.u & 1][sgm - G.shared_on], 0), G.E - 1) *
+                                L.expert_stride;
+      const uint8_t* dn = eb + 2 * G.q_gu;
+      if ((q & 1) == 0) {
+        *src = dn + (size_t)cv.r0 * G.rc_i;
+        *dst_off = (unsigned)sgm * G.Rd * G.rc_i;
+        return (unsigned)cv.n * G.rc_i;
+      }
+      *src = dn + (size_t)G.H * G.rc_i + (size_t)cv.r0 * G.rs_i;
+      *dst_off = (unsigned)G.nseg * G.Rd * G.rc_i + (unsigned)sgm * G.Rd * G.rs_i;
+      return (unsigned)cv.n * G.rs_i;
+    }
+  }
+}
+
+// Bulk copies a chunk takes (some may be empty, see copy_desc) and its total bytes.
+__device__ __forceinline__ int copies_of(const Geo& G, const Chunk& cv) {
+  return cv.kind == K_ROUTER ? (G.rseg == 1 ? 2 : 1) : (cv.kind == K_DN ? 2 * G.nseg : 4);
+}
+
+__device__ __forceinline__ unsigned chunk_bytes(const Geo& G, const Chunk& cv) {
+  switch (cv.kind) {
+    case K_ROUTER:
+      if (G.rseg > 1) return 4u * (unsigned)G.rcols;
+      return (unsigned)cv.n * 4u * (unsigned)G.H;  // router rows and the gate row alike
+    case K_SGU:
+    case K_RGU:
+      return 2u * (unsigned)cv.n * (G.rc_h + G.rs_h);
+    default:
+      return (unsigned)G.nseg * (unsigned)cv.n * (G.rc_i + G.rs_i);
+  }
+}
+
+// The whole producer warp walks this CTA's chunks in order, several chunks per step: the
+// lanes are dealt out to the copies of consecutive chunks (at most 8 chunks, 32 copies), the
+// first lane of each chunk waits for its stage to be free and registers the chunk's bytes on
+// the stage's barrier, then every lane issues its copy. Routed chunks of a unit wait, once,
+// for the CTA's routing decision of that unit; a step never spans that wait.
 __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
+  const int lane = threadIdx.x & 31;
   const unsigned NS = (unsigned)G.nstage;
   const unsigned n_local = local_chunks(P, G);
-  int rt_u = -1;
-  int eidx[kMaxK];
-#pragma unroll
-  for (int k = 0; k < kMaxK; ++k) eidx[k] = 0;
+  int rt_u = -1;  // unit whose routing decision this warp has seen
+  ChunkWalk cw;
+  cw.init(G, blockIdx.x, (int)gridDim.x);
   unsigned i = 0;
-  for (; i < n_local; ++i) {
-    const int slot = (int)(i % NS);
-    if (!wait_mbar(P, sm, &empty[slot], ((i / NS) & 1u) ^ 1u, DE_TIMEOUT_EMPTY)) break;
-    const Chunk cv =
-        chunk_at(G, (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x);
-    const bool routed = cv.kind == K_RGU || (cv.kind == K_DN && G.routed_on);
-    if (routed && cv.u != rt_u) {
-      if (wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(cv.u + 1), DE_TIMEOUT_ROUTE) == 0u)
-        break;
-      for (int k = 0; k < G.K; ++k) eidx[k] = min(max(sm->rt_e[cv.u & 1][k], 0), G.E - 1);
-      rt_u = cv.u;
-    }
-    const LayerW& L = P.layers[cv.u % P.n_layers];
-    uint8_t* dst = smem + G.o_ring + (size_t)slot * G.stage_bytes;
-    switch (cv.kind) {
-      case K_ROUTER: {
-        if (G.rseg == 1) {  // whole rows r0 .. r0+n-1; row E is the shared-gate vector
-          const unsigned rowb = 4u * (unsigned)G.H;
-          const int a = cv.r0, b = min(cv.r0 + cv.n, G.E);
-          const bool gate_row = cv.r0 + cv.n > G.E;
-          const unsigned bytes = (b > a ? (unsigned)(b - a) * rowb : 0u) + (gate_row ? rowb : 0u);
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          if (b > a)
-            copy_rows(dst, reinterpret_cast<const uint8_t*>(L.router + (size_t)a * G.H),
-                      (unsigned)(b - a) * rowb, &full[slot]);
-          if (gate_row)
-            copy_rows(dst + (size_t)(G.E - cv.r0) * rowb, reinterpret_cast<const uint8_t*>(L.gate),
-                      rowb, &full[slot]);
-        } else {  // one column segment of row r0
-          const float* row = cv.r0 < G.E ? L.router + (size_t)cv.r0 * G.H : L.gate;
-          const unsigned bytes = 4u * (unsigned)G.rcols;
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          copy_rows(dst, reinterpret_cast<const uint8_t*>(row + (size_t)cv.seg * G.rcols), bytes,
-                    &full[slot]);
+  bool failed = false;
+  while (i < n_local) {
+    // routing of the first chunk's unit, if it is routed and new
+    {
+      const Chunk c0 = chunk_view(G, cw.u, cw.c);
+      if ((c0.kind == K_RGU || (c0.kind == K_DN && G.routed_on)) && c0.u != rt_u) {
+        int ok = 1;
+        if (lane == 0)
+          ok = wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(c0.u + 1),
+                          DE_TIMEOUT_ROUTE) != 0u;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          failed = true;
+          break;
         }
-        break;
-      }
-      case K_SGU:
-      case K_RGU: {  // stage: gate codes | up codes | gate sb | up sb, R rows each
-        const uint8_t* base =
-            cv.kind == K_SGU ? L.shared : L.experts + (size_t)eidx[cv.k] * L.expert_stride;
-        const unsigned cb = (unsigned)cv.n * G.rc_h, sbb = (unsigned)cv.n * G.rs_h;
-        mbar_arrive_expect_tx(&full[slot], 2u * (cb + sbb));
-        const size_t sbo = (size_t)G.I * G.rc_h;
-        copy_rows(dst, base + (size_t)cv.r0 * G.rc_h, cb, &full[slot]);
-        copy_rows(dst + (size_t)G.R * G.rc_h, base + G.q_gu + (size_t)cv.r0 * G.rc_h, cb,
-                  &full[slot]);
-        uint8_t* dsb = dst + (size_t)2 * G.R * G.rc_h;
-        copy_rows(dsb, base + sbo + (size_t)cv.r0 * G.rs_h, sbb, &full[slot]);
-        copy_rows(dsb + (size_t)G.R * G.rs_h, base + G.q_gu + sbo + (size_t)cv.r0 * G.rs_h, sbb,
-                  &full[slot]);
-        break;
-      }
-      default: {  // K_DN: per segment (shared first, then routed k) Rd rows of codes | sb
-        const unsigned cb = (unsigned)cv.n * G.rc_i, sbb = (unsigned)cv.n * G.rs_i;
-        mbar_arrive_expect_tx(&full[slot], (unsigned)G.nseg * (cb + sbb));
-        uint8_t* dsb = dst + (size_t)G.nseg * G.Rd * G.rc_i;
-        for (int s = 0; s < G.nseg; ++s) {
-          const uint8_t* eb = (G.shared_on && s == 0)
-                                  ? L.shared
-                                  : L.experts + (size_t)eidx[s - G.shared_on] * L.expert_stride;
-          const uint8_t* dn = eb + 2 * G.q_gu;
-          copy_rows(dst + (size_t)s * G.Rd * G.rc_i, dn + (size_t)cv.r0 * G.rc_i, cb, &full[slot]);
-          copy_rows(dsb + (size_t)s * G.Rd * G.rs_i,
-                    dn + (size_t)G.H * G.rc_i + (size_t)cv.r0 * G.rs_i, sbb, &full[slot]);
-        }
-        break;
+        __syncwarp();
+        rt_u = c0.u;
       }
     }
-    sm->issued = i + 1;
+    // deal the lanes out to the copies of the next chunks (the same plan in every lane)
+    Chunk my{};
+    int my_q = -1;
+    unsigned my_i = 0;
+    int nb = 0, used = 0;
+    ChunkWalk w = cw;
+    while (nb < 8 && i + (unsigned)nb < n_local) {
+      const Chunk c = chunk_view(G, w.u, w.c);
+      if ((c.kind == K_RGU || (c.kind == K_DN && G.routed_on)) && c.u != rt_u) break;
+      const int nc = copies_of(G, c);
+      if (used + nc > 32) break;
+      if (lane >= used && lane < used + nc) {
+        my = c;
+        my_q = lane - used;
+        my_i = i + (unsigned)nb;
+      }
+      used += nc;
+      ++nb;
+      w.next();
+    }
+    // stages free?
+    int ok = 1;
+    if (my_q == 0)
+      ok = wait_mbar(P, sm, &empty[my_i % NS], ((my_i / NS) & 1u) ^ 1u, DE_TIMEOUT_EMPTY);
+    if (!__all_sync(0xffffffffu, ok)) {
+      failed = true;
+      break;
+    }
+    if (my_q == 0) mbar_arrive_expect_tx(&full[my_i % NS], chunk_bytes(G, my));
+    __syncwarp();
+    if (my_q >= 0) {
+      const LayerW& L = P.layers[my.u % P.n_layers];
+      const uint8_t* src = nullptr;
+      unsigned dst_off = 0;
+      const unsigned bytes = copy_desc(G, L, sm, my, my_q, &src, &dst_off);
+      if (bytes)
+        tma_load_1d(smem + G.o_ring + (size_t)(my_i % NS) * G.stage_bytes + dst_off, src, bytes,
+                    &full[my_i % NS]);
+    }
+    __syncwarp();
+    i += (unsigned)nb;
+    cw = w;
   }
   // never leave the CTA with bulk copies in flight: wait for the last copies of every stage
-  if (i < n_local) {
+  if (lane == 0 && failed) {
     const uint64_t deadline = global_ns() + 100000000ull;
     const unsigned first = i > NS ? i - NS : 0u;
     for (unsigned j = first; j < i; ++j) {
-      const int s = (int)(j % NS);
-      while (!mbar_try_wait(&full[s], (j / NS) & 1u)) {
+      const int st = (int)(j % NS);
+      while (!mbar_try_wait(&full[st], (j / NS) & 1u)) {
         if (global_ns() > deadline) {
           atomicCAS(P.s.err, 0, DE_TIMEOUT_DRAIN);
           return;
@@ -1034,11 +1132,13 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
   UnitView uv;
   unsigned x_seen = 0, xd_seen = 0;  // units known ready (counter values already acquired)
   unsigned mine = 0;                 // chunks of the current run done by this warp
-  for (unsigned i = (unsigned)w; i < n_local; i += kConsumerWarps) {
+  ChunkWalk cw;
+  cw.init(G, (unsigned long long)blockIdx.x + (unsigned long long)w * gridDim.x,
+          kConsumerWarps * (int)gridDim.x);
+  for (unsigned i = (unsigned)w; i < n_local; i += kConsumerWarps, cw.next()) {
     const int slot = (int)(i % NS);
     if (!warp_wait_mbar(P, sm, &full[slot], (i / NS) & 1u, DE_TIMEOUT_FULL)) break;
-    const unsigned long long g = (unsigned long long)blockIdx.x + (unsigned long long)i * gridDim.x;
-    const Chunk cv = chunk_at(G, g);
+    const Chunk cv = chunk_view(G, cw.u, cw.c);
     if (cv.u != cur_u) {
       cur_u = cv.u;
       uv = unit_view(P, G, cv.u);
@@ -1065,8 +1165,9 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
     const int cls = class_of(cv.kind);
     bool run_end = i + kConsumerWarps >= n_local;
     if (!run_end) {
-      const Chunk nx = chunk_at(G, g + (unsigned long long)kConsumerWarps * gridDim.x);
-      run_end = nx.u != cv.u || class_of(nx.kind) != cls;
+      ChunkWalk nw = cw;
+      nw.next();
+      run_end = nw.u != cv.u || class_of(chunk_view(G, nw.u, nw.c).kind) != cls;
     }
     if (run_end) {
       finish_run(P, G, sm, cls, cv.u, mine);
@@ -1084,7 +1185,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     sm->abort = 0;
     for (int c = 0; c < CL_COUNT; ++c) sm->run_cnt[c] = 0;
-    sm->issued = 0;
     sm->x_ready = sm->rt_ready = sm->xd_ready = 0;
     mbar_init(&sm->x_bar, 1);
     mbar_init(&sm->rt_bar, 1);
@@ -1099,7 +1199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) producer(P, G, smem, sm);
+    producer(P, G, smem, sm);
     return;
   }
   if (warp == 1) {
