@@ -606,14 +606,19 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
 #pragma unroll
   for (int i = 0; i < kPer; ++i) best[i] = 0ull;
   for (int e0 = 0; e0 < G.E; e0 += 32 * kPer) {
-    // all loads of a segment are independent, so each segment costs one round trip
-    double lv[kPer];
+    // the bias and the first two segments' partials are loaded together (one round trip)
+    double lv[kPer], p1[kPer];
+    float bv[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int ec = min(e0 + lane + 32 * i, G.E - 1);
-      lv[i] = bias ? (double)__ldcg(bias + ec) : 0.0;
+      bv[i] = bias ? __ldcg(bias + ec) : 0.f;
+      lv[i] = __ldcg(lg + ec);
+      p1[i] = G.rseg > 1 ? __ldcg(lg + (size_t)G.nr + ec) : 0.0;
     }
-    for (int s = 0; s < G.rseg; ++s) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) lv[i] = ((double)bv[i] + lv[i]) + p1[i];
+    for (int s = 2; s < G.rseg; ++s) {
       double part[kPer];
 #pragma unroll
       for (int i = 0; i < kPer; ++i)
@@ -717,6 +722,7 @@ __device__ __forceinline__ void transform_slices(float* raw, float* xt, float* s
                                                  int bits, ScaleOf scale_of,
                                                  bool write_back_raw) {
   const int lane = threadIdx.x & 31;
+#pragma unroll 4
   for (int t = lane; t < nsl; t += 32) {
     const float f = scale_of(t);
     float4 v[8];
