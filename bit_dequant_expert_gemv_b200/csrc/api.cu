@@ -218,8 +218,10 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   G->o_misc = take(512);
   const unsigned fixed = o;
   const unsigned avail = (unsigned)max_smem;
-  if (fixed + 2 * (G->stage_bytes + 16) > avail)
-    return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for two stages");
+  // at least one stage per consumer warp: the first chunks of a unit that need a shared
+  // transform (one per warp) must all fit in the ring at once
+  if (fixed + kConsumerWarps * (G->stage_bytes + 16) > avail)
+    return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for %d stages", kConsumerWarps);
   int ns = (int)((avail - fixed) / (G->stage_bytes + 16));
   ns = std::min(ns, kMaxStages);
   G->nstage = ns;

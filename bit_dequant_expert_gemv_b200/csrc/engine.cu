@@ -197,10 +197,16 @@ struct Smem {  // small shared state (in the misc area)
   // Readiness per unit: a monotone counter (units ready so far; the truth) and an mbarrier
   // that completes one phase per unit, used only to sleep until the next increment. Waiters
   // may run several units ahead of the stager, so the counter decides, never the parity.
-  uint64_t x_bar;              // x staged
+  uint64_t x_bar;              // raw x of the unit in XA (the router's input)
   uint64_t rt_bar;             // routing decision in rt_e / rt_w
-  uint64_t xd_bar;             // down input staged
+  uint64_t xd_bar;             // raw down input [h_s | h_k] of the unit in XA
   unsigned x_ready, rt_ready, xd_ready;
+  // The transforms of x (into XG) and of the down input (in place in XA) are shared by the
+  // consumer warps: one eighth each (the stager does the eighths of warps that have no chunk
+  // needing them); per unit parity, the number of slices transformed so far.
+  unsigned xg_done[2], xd_done[2];
+  float xf[2];                 // RMSNorm factor of the unit's x (1 without a norm)
+  float sigma[2];              // sigmoid(g . x) of the unit (1 without a shared gate)
   volatile int abort;
   unsigned run_cnt[CL_COUNT];  // chunks of the current run of each class finished here
   int rt_e[2][kMaxK];          // routing of unit u (index u & 1): experts and weights
@@ -280,6 +286,22 @@ __device__ __noinline__ unsigned wait_ready(const Prog& P, Smem* sm, const unsig
   }
 }
 
+// Wait until the shared counter *cnt reaches target (a few warps' transform shares away).
+__device__ __noinline__ bool wait_count(const Prog& P, Smem* sm, const unsigned* cnt,
+                                        unsigned target, int code) {
+  if (ld_acquire_cta_smem(cnt) >= target) return true;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_cta_smem(cnt) >= target) return true;
+    if (sm->abort) return false;
+    if (global_ns() > deadline) {
+      raise_error(P, sm, code);
+      return false;
+    }
+  }
+}
+
 // the stager's side: publish "unit u is ready" on a counter and wake sleepers
 __device__ __forceinline__ void signal_ready(unsigned* cnt, uint64_t* bar, int u) {
   st_release_cta_smem(cnt, (unsigned)(u + 1));
@@ -305,6 +327,15 @@ __device__ __forceinline__ unsigned warp_wait_ready(const Prog& P, Smem* sm, con
   c = __shfl_sync(0xffffffffu, c, 0);
   __syncwarp();
   return c;
+}
+
+__device__ __forceinline__ bool warp_wait_count(const Prog& P, Smem* sm, const unsigned* cnt,
+                                                unsigned target, int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_count(P, sm, cnt, target, code);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
 }
 
 __device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t* bar,
@@ -335,7 +366,6 @@ __device__ __forceinline__ void finish_run(const Prog& P, const Geo& G, Smem* sm
     const unsigned nrun = run_len(G, u, cls);
     if (old + mine == nrun) {
       atom_exch_cta_smem(&sm->run_cnt[cls], 0u);
-      fence_acq_rel_gpu();
       const unsigned og = atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cls), nrun);
       bcast = og + nrun == (unsigned)(u + 1) * (unsigned)G.ncl[cls];
     }
@@ -632,37 +662,47 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
       const int e = e0 + lane + 32 * i;
       key[i] = e < G.E ? pkey(lv[i], e) : 0ull;
     }
-    sort16_desc(key);
-    if (e0 == 0) {
+    if (G.E <= 32 * kPer) {  // one block: the lane's 16 keys are its candidates, unsorted
 #pragma unroll
       for (int i = 0; i < kPer; ++i) best[i] = key[i];
     } else {
-      // both lists sorted descending: best[i] vs key[15-i] keeps the 16 largest as a bitonic
-      // sequence, which one more sort puts in order
+      // keep each lane's 16 largest keys: both lists sorted descending, best[i] vs key[15-i]
+      // is a bitonic sequence holding the 16 largest, which one more sort puts in order
+      sort16_desc(key);
+      if (e0 == 0) {
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) best[i] = umax64(best[i], key[kPer - 1 - i]);
-      sort16_desc(best);
+        for (int i = 0; i < kPer; ++i) best[i] = key[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) best[i] = umax64(best[i], key[kPer - 1 - i]);
+        sort16_desc(best);
+      }
     }
   }
+  // K rounds: the warp maximum of the lanes' largest candidates (two 32-bit reductions); the
+  // lane that held it drops it and finds its next largest
+  unsigned long long m = 0ull;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) m = umax64(m, best[i]);
   int sel_e = 0;  // lane k < K ends up holding winner k
   unsigned long long sel_k = 0ull;
+  for (int k = 0; k < G.K; ++k) {
+    const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(m >> 32));
+    const unsigned lo =
+        __reduce_max_sync(0xffffffffu, (unsigned)(m >> 32) == hi ? (unsigned)m : 0u);
+    const unsigned long long win = ((unsigned long long)hi << 32) | lo;
+    if (m == win && win != 0ull) {
+      unsigned long long nm = 0ull;
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
-    if (k < G.K) {
-      const unsigned long long head = best[0];
-      const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(head >> 32));
-      const unsigned lo =
-          __reduce_max_sync(0xffffffffu, (unsigned)(head >> 32) == hi ? (unsigned)head : 0u);
-      const unsigned long long win = ((unsigned long long)hi << 32) | lo;
-      if (head == win && win != 0ull) {
-#pragma unroll
-        for (int j = 0; j + 1 < kMaxK; ++j) best[j] = best[j + 1];
-        best[kMaxK - 1] = 0ull;
+      for (int i = 0; i < kPer; ++i) {
+        best[i] = best[i] == win ? 0ull : best[i];
+        nm = umax64(nm, best[i]);
       }
-      if (lane == k) {
-        sel_k = win;
-        sel_e = 0x1FFF - (int)(win & 0x1FFFull);
-      }
+      m = nm;
+    }
+    if (lane == k) {
+      sel_k = win;
+      sel_e = 0x1FFF - (int)(win & 0x1FFFull);
     }
   }
   const double l0 = dkey_inv(__shfl_sync(0xffffffffu, sel_k, 0) & ~0x1FFFull);
@@ -714,37 +754,55 @@ __device__ __forceinline__ bool stage_in(const Prog& P, Smem* sm, void* dst, con
   return ok;
 }
 
-// Transform nsl slices of raw values in `raw` (linear layout) into `xt` (swizzled) and their
-// sums into `sx`; slice t is scaled by scale_of(t) first (and written back to `raw` when
-// asked). raw and xt may be the same array: a slice is read whole before it is written.
+// Share w (of 8) of a transform: slices [w*nsl/8, (w+1)*nsl/8) of the raw values in `raw`
+// (linear layout) go into `xt` (swizzled) with their sums in `sx`, slice t scaled by
+// scale_of(t) first. One lane per slice (consecutive slices: the swizzle keeps each
+// quarter-warp on distinct banks); raw and xt may be the same array (a lane reads its whole
+// slice before it writes it). Returns the number of slices done.
 template <typename ScaleOf>
-__device__ __forceinline__ void transform_slices(float* raw, float* xt, float* sx, int nsl,
-                                                 int bits, ScaleOf scale_of,
-                                                 bool write_back_raw) {
+__device__ __forceinline__ int transform_share(const float* raw, float* xt, float* sx, int nsl,
+                                               int w, int bits, ScaleOf scale_of) {
   const int lane = threadIdx.x & 31;
-#pragma unroll 4
-  for (int t = lane; t < nsl; t += 32) {
+  const int t0 = w * nsl / 8, t1 = (w + 1) * nsl / 8;
+  for (int t = t0 + lane; t < t1; t += 32) {
     const float f = scale_of(t);
     float4 v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {  // v[i] = logical float4 q = i ^ (t & 7): distinct banks
-      const int q = i ^ (t & 7);
-      v[i] = *reinterpret_cast<const float4*>(raw + 32 * t + 4 * q);
+      v[i] = *reinterpret_cast<const float4*>(raw + 32 * t + 4 * (i ^ (t & 7)));
       v[i].x *= f; v[i].y *= f; v[i].z *= f; v[i].w *= f;
     }
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-    if (write_back_raw) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<float4*>(raw + 32 * t + 4 * (i ^ (t & 7))) = v[i];
-    }
+    for (int i = 0; i < 8; ++i) sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
 #pragma unroll
     for (int i = 0; i < 8; ++i)  // logical q = i ^ (t & 7) belongs at xpos(t, q) = 32t + 4i
       *reinterpret_cast<float4*>(xt + 32 * t + 4 * i) = xform(v[i], bits);
-    sx[t] = s;
+    sx[t] = sum;
   }
+  __syncwarp();
+  return t1 - t0;
+}
+
+// Local index range [lo, hi) of this CTA's chunks with unit index in [u*ntot + c0, u*ntot + c1).
+__device__ __forceinline__ void local_range(const Geo& G, int u, int c0, int c1, unsigned* lo,
+                                            unsigned* hi) {
+  const unsigned long long base = (unsigned long long)u * (unsigned)G.off[K_COUNT];
+  *lo = count_cong(0ull, base + (unsigned)c0, blockIdx.x, gridDim.x);
+  *hi = *lo + count_cong(base + (unsigned)c0, base + (unsigned)c1, blockIdx.x, gridDim.x);
+}
+
+// Does consumer warp w get a chunk with local index in [lo, hi)? (local chunk i -> warp i mod 8)
+__device__ __forceinline__ bool warp_in_range(unsigned lo, unsigned hi, int w) {
+  const unsigned cnt = hi - lo;
+  return cnt >= (unsigned)kConsumerWarps ||
+         ((unsigned)(w - (int)(lo % kConsumerWarps) + kConsumerWarps) % kConsumerWarps) < cnt;
+}
+
+// The scale of down-input slice t: sigma for the shared expert's segment, w_k for routed k.
+__device__ __forceinline__ float xd_scale(const Geo& G, const Smem* sm, int u, int t) {
+  const int s = t / (G.I / 32);
+  return (G.shared_on && s == 0) ? sm->sigma[u & 1] : sm->rt_w[u & 1][s - G.shared_on];
 }
 
 __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
@@ -757,6 +815,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   const unsigned ntot = (unsigned)G.off[K_COUNT];
   const bool gu_on = G.shared_on || G.routed_on;
   unsigned xphase = 0;
+  (void)lane;
   for (int u = 0; u < P.n_units; ++u) {
     const UnitView uv = unit_view(P, G, u);
     const bool owner = ((unsigned long long)u * ntot) % gridDim.x == blockIdx.x;
@@ -768,19 +827,23 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     if (owner && uv.h_trace)
       for (int c = lane * 4; c < G.H; c += 128)
         *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XA + c);
-    __syncwarp();  // every lane has read the raw x before any lane rescales it in place
-    if (gu_on) {
-      transform_slices(XA, XG, SXG, G.H / 32, G.bits, [&](int) { return f; },
-                       G.route_on && uv.norm);
-    } else if (uv.norm) {
-      for (int c = lane * 4; c < G.H; c += 128) {
-        float4 v = *reinterpret_cast<float4*>(XA + c);
-        v.x *= f; v.y *= f; v.z *= f; v.w *= f;
-        *reinterpret_cast<float4*>(XA + c) = v;
-      }
+    if (lane == 0) {
+      sm->xf[u & 1] = f;
+      sm->xg_done[u & 1] = 0u;
     }
     __syncwarp();
     if (lane == 0) signal_ready(&sm->x_ready, &sm->x_bar, u);
+    // the eighths of the x transform that no consumer warp will do (warps without a gate/up
+    // chunk of this unit)
+    if (gu_on) {
+      unsigned lo, hi;
+      local_range(G, u, G.off[K_SGU], G.off[K_DN], &lo, &hi);
+      int done = 0;
+      for (int w = 0; w < kConsumerWarps; ++w)
+        if (!warp_in_range(lo, hi, w))
+          done += transform_share(XA, XG, SXG, G.H / 32, w, G.bits, [&](int) { return f; });
+      if (done && lane == 0) red_release_cta_smem(&sm->xg_done[u & 1], (unsigned)done);
+    }
     // ---- routing decision: needs every router chunk of unit u
     float sigma = 1.f;
     if (G.route_on) {
@@ -788,6 +851,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
       if (G.gate_on)  // sigma(g . x): the shared-gate row is router row E
         sigma = (float)(1.0 / (1.0 + exp(-unit_logit(G, lg, G.E))));
+      if (lane == 0) sm->sigma[u & 1] = sigma;
       topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
                 owner ? uv.w_out : nullptr);
       __syncwarp();
@@ -798,20 +862,24 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       if (!warp_wait_flag(P, sm, CL_GU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
       const unsigned bs = G.shared_on ? 4u * (unsigned)G.I : 0u;
       const unsigned bk = G.routed_on ? 4u * (unsigned)(G.K * G.I) : 0u;
+      if (lane == 0) {
+        sm->xd_done[u & 1] = 0u;
+        if (!G.route_on) sm->sigma[u & 1] = 1.f;
+      }
       if (!stage_in(P, sm, XA, P.s.hs + (size_t)uv.slot * G.I, bs, xphase,
                     XA + (size_t)G.shared_on * G.I, P.s.hk + (size_t)uv.slot * G.K * G.I, bk))
         break;
-      const int spseg = G.I / 32;
-      const float* rw = sm->rt_w[u & 1];
-      transform_slices(
-          XA, XA, SXA, G.nseg * spseg, G.bits,
-          [&](int t) {
-            const int s = t / spseg;
-            return (G.shared_on && s == 0) ? sigma : rw[s - G.shared_on];
-          },
-          false);
       __syncwarp();
       if (lane == 0) signal_ready(&sm->xd_ready, &sm->xd_bar, u);
+      // the eighths of the down-input transform that no consumer warp will do
+      unsigned lo, hi;
+      local_range(G, u, G.off[K_DN], G.off[K_COUNT], &lo, &hi);
+      int done = 0;
+      for (int w = 0; w < kConsumerWarps; ++w)
+        if (!warp_in_range(lo, hi, w))
+          done += transform_share(XA, XA, SXA, G.nseg * (G.I / 32), w, G.bits,
+                                  [&](int t) { return xd_scale(G, sm, u, t); });
+      if (done && lane == 0) red_release_cta_smem(&sm->xd_done[u & 1], (unsigned)done);
     }
   }
 }
@@ -1009,7 +1077,7 @@ __device__ __forceinline__ void release_stage(uint64_t* empty) {
 // router rows r0..r0+n-1, columns seg*rcols .. +rcols: binary64 sums of fp32 products
 __device__ __forceinline__ void router_chunk(const Prog& P, const Geo& G, const Chunk& cv,
                                              const uint8_t* stage, uint64_t* empty,
-                                             const float* XR) {
+                                             const float* XR, float xf) {
   const int lane = threadIdx.x & 31;
   const float4* xr = reinterpret_cast<const float4*>(XR + (size_t)cv.seg * G.rcols);
   const int nf = G.rcols / 4;
@@ -1028,7 +1096,7 @@ __device__ __forceinline__ void router_chunk(const Prog& P, const Geo& G, const 
     double a = (a0 + a1) + (a2 + a3);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == (r & 31)) res = a;
+    if (lane == (r & 31)) res = a * (double)xf;  // the norm factor of x, applied to the sum
     if ((r & 31) == 31 || r == cv.n - 1) {  // flush up to 32 results, one per lane
       const int rb = r & ~31;
       if (lane <= (r & 31)) lg[rb + lane] = res;
@@ -1131,37 +1199,68 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
   float* red = reinterpret_cast<float*>(smem + G.o_red) + (size_t)w * 16 * kRowsPerLane;
-  const float* XR = reinterpret_cast<const float*>(smem + G.o_xa);
+  float* XA = reinterpret_cast<float*>(smem + G.o_xa);
+  float* SXA = reinterpret_cast<float*>(smem + G.o_sxa);
+  float* XG = reinterpret_cast<float*>(smem + G.o_xg);
+  float* SXG = reinterpret_cast<float*>(smem + G.o_sxg);
+  const int lane = threadIdx.x & 31;
   const unsigned NS = (unsigned)G.nstage;
   const unsigned n_local = local_chunks(P, G);
   int cur_u = -1;
   UnitView uv;
   unsigned x_seen = 0, xd_seen = 0;  // units known ready (counter values already acquired)
+  unsigned xg_mine = 0, xd_mine = 0; // units (+1) whose transform share this warp has done
   unsigned mine = 0;                 // chunks of the current run done by this warp
   ChunkWalk cw;
   cw.init(G, (unsigned long long)blockIdx.x + (unsigned long long)w * gridDim.x,
           kConsumerWarps * (int)gridDim.x);
   for (unsigned i = (unsigned)w; i < n_local; i += kConsumerWarps, cw.next()) {
     const int slot = (int)(i % NS);
-    if (!warp_wait_mbar(P, sm, &full[slot], (i / NS) & 1u, DE_TIMEOUT_FULL)) break;
     const Chunk cv = chunk_view(G, cw.u, cw.c);
     if (cv.u != cur_u) {
       cur_u = cv.u;
       uv = unit_view(P, G, cv.u);
     }
     const unsigned need = (unsigned)(cv.u + 1);
+    // the input of the chunk; at the warp's first chunk of the unit that needs a transformed
+    // input, its share of the transform, done before the chunk's weights are waited for
+    bool share_wait = false;
     if (cv.kind == K_DN) {
       if ((int)(xd_seen - need) < 0) {
         xd_seen = warp_wait_ready(P, sm, &sm->xd_ready, &sm->xd_bar, need, DE_TIMEOUT_DEP);
         if (xd_seen == 0u) break;
       }
-    } else if ((int)(x_seen - need) < 0) {
-      x_seen = warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, need, DE_TIMEOUT_DEP);
-      if (x_seen == 0u) break;
+      if (xd_mine != need) {
+        xd_mine = need;
+        share_wait = true;
+        const int d = transform_share(XA, XA, SXA, G.nseg * (G.I / 32), w, G.bits,
+                                      [&](int t) { return xd_scale(G, sm, cv.u, t); });
+        if (lane == 0 && d) red_release_cta_smem(&sm->xd_done[cv.u & 1], (unsigned)d);
+      }
+    } else {
+      if ((int)(x_seen - need) < 0) {
+        x_seen = warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, need, DE_TIMEOUT_DEP);
+        if (x_seen == 0u) break;
+      }
+      if (cv.kind != K_ROUTER && xg_mine != need) {
+        xg_mine = need;
+        share_wait = true;
+        const float f = sm->xf[cv.u & 1];
+        const int d = transform_share(XA, XG, SXG, G.H / 32, w, G.bits,
+                                      [&](int) { return f; });
+        if (lane == 0 && d) red_release_cta_smem(&sm->xg_done[cv.u & 1], (unsigned)d);
+      }
+    }
+    if (!warp_wait_mbar(P, sm, &full[slot], (i / NS) & 1u, DE_TIMEOUT_FULL)) break;
+    if (share_wait) {  // every other share of the transform
+      const bool dn = cv.kind == K_DN;
+      if (!warp_wait_count(P, sm, dn ? &sm->xd_done[cv.u & 1] : &sm->xg_done[cv.u & 1],
+                           (unsigned)(dn ? G.nseg * (G.I / 32) : G.H / 32), DE_TIMEOUT_DEP))
+        break;
     }
     const uint8_t* stage = smem + G.o_ring + (size_t)slot * G.stage_bytes;
     if (cv.kind == K_ROUTER)
-      router_chunk(P, G, cv, stage, &empty[slot], XR);
+      router_chunk(P, G, cv, stage, &empty[slot], XA, sm->xf[cv.u & 1]);
     else if (G.bits == 4)
       dispatch_dot<4>(P, G, cv, uv, stage, &empty[slot], smem, red);
     else
