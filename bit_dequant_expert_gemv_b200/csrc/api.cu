@@ -257,16 +257,15 @@ int check_layer(const fmoe_layer_desc* L, const fmoe_layer_desc* L0) {
 
 // ---------------------------------------------------------------- scratch
 struct ScratchPlan {
-  size_t off_ctrl, off_flags, off_normsq, zero_bytes, off_logits, off_hs, off_hk, off_hbuf, total;
+  size_t off_ctrl, off_normsq, zero_bytes, off_logits, off_hs, off_hk, off_hbuf, total;
 };
 
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
-ScratchPlan plan_scratch(const Geo& G, int n_units, int max_grid) {
+ScratchPlan plan_scratch(const Geo& G, int n_units) {
   ScratchPlan s;
   size_t o = 0;
   s.off_ctrl = o; o = up256(o + 4 * C_WORDS);
-  s.off_flags = o; o = up256(o + 4 * (size_t)F_WORDS * max_grid);
   s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
   s.zero_bytes = o;
   s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.rseg, 1) * std::max(G.nr, 1));
@@ -279,7 +278,6 @@ ScratchPlan plan_scratch(const Geo& G, int n_units, int max_grid) {
 
 void bind_scratch(Prog* P, const ScratchPlan& sp, uint8_t* base, int* err) {
   P->s.ctrl = reinterpret_cast<unsigned*>(base + sp.off_ctrl);
-  P->s.flags = reinterpret_cast<unsigned*>(base + sp.off_flags);
   P->s.normsq = reinterpret_cast<float*>(base + sp.off_normsq);
   P->s.logits = reinterpret_cast<double*>(base + sp.off_logits);
   P->s.hs = reinterpret_cast<float*>(base + sp.off_hs);
@@ -312,7 +310,7 @@ int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, 
 
 // Run a program with scratch taken from the library's stream-ordered pool.
 int run_pooled(Prog* P, const Geo& G, DevState* d, cudaStream_t st) {
-  const ScratchPlan sp = plan_scratch(G, P->n_units, d->sms);
+  const ScratchPlan sp = plan_scratch(G, P->n_units);
   void* base = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&base, sp.total, d->pool, st);
   if (e != cudaSuccess) return fail(FMOE_ERR_NOMEM, "scratch allocation: %s", cudaGetErrorString(e));
@@ -605,7 +603,7 @@ int fmoe_moe_layer_noalloc(const fmoe_layer_desc* layer, const float* x, const f
   if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
     return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
   if (x == out) return fail(FMOE_ERR_INVALID, "x must not alias out");
-  const ScratchPlan sp = plan_scratch(G, 1, s->sms);
+  const ScratchPlan sp = plan_scratch(G, 1);
   if (sp.total > kNoAllocErrOff)
     return fail(FMOE_ERR_UNSUPPORTED,
                 "fmoe_moe_layer_noalloc: this shape needs %zu bytes of scratch, the fixed area "
@@ -683,7 +681,7 @@ int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const f
   if (tokens_per_launch <= 0 || tokens_per_launch > n_tokens) tokens_per_launch = n_tokens;
   const int H = G.H, E = G.E, K = G.K, L = n_layers;
   const int units_per_launch = tokens_per_launch * L;
-  const ScratchPlan sp = plan_scratch(G, units_per_launch, d->sms);
+  const ScratchPlan sp = plan_scratch(G, units_per_launch);
   fmoe_graph* g = new fmoe_graph();
   cudaError_t e = cudaMalloc(&g->scratch, sp.total);
   if (e != cudaSuccess) {

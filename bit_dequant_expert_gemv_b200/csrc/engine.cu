@@ -28,11 +28,11 @@
 //                   arithmetic, reduces its row sums inside the warp and runs the chunk's
 //                   epilogue (logit store, SwiGLU, or residual + combine) itself -- no
 //                   block-wide barrier and no cross-warp reduction on the hot path.
-// Completion is published per run of same-class chunks of a CTA: the warp finishing a run's
-// last chunk makes one gpu-scope fence and one atomic, and the CTA completing a class for a
-// unit writes a flag into every CTA's own flag line. Every spin-wait is bounded by a
-// global-timer budget; on expiry the kernel records an error word, waits for its own copies
-// in flight and returns.
+// Completion is counted per run of same-class chunks of a CTA: the warp finishing a CTA's run
+// makes one gpu-scope release-acquire atomic on the class counter, and the stager warps poll
+// that counter (it is performed in L2, so no second hop is needed). Every spin-wait is
+// bounded by a global-timer budget; on expiry the kernel records an error word, waits for
+// its own copies in flight and returns.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -42,10 +42,6 @@
 namespace fmoe {
 
 __device__ __forceinline__ int cnt_word(int cls) { return C_CNT + 32 * cls; }
-// this CTA's flag word `w` (units whose class w is complete)
-__device__ __forceinline__ const unsigned* my_flag(const Prog& P, int w) {
-  return P.s.flags + blockIdx.x * F_WORDS + w;
-}
 
 // ------------------------------------------------------------------------------------------
 // unit and chunk views
@@ -218,8 +214,8 @@ __device__ __forceinline__ void raise_error(const Prog& P, Smem* sm, int code) {
   sm->abort = 1;
 }
 
-// Spin until *a - target >= 0 (wrap-safe) on a gpu-scope flag, the budget runs out, the CTA
-// aborts or another CTA has recorded an error.
+// Spin until *a - target >= 0 (wrap-safe) on a gpu-scope counter, the budget runs out, the
+// CTA aborts or another CTA has recorded an error.
 // Polls with relaxed loads (an acquire per poll would be a gpu-scope ordering operation each
 // time) and makes one acquire fence once the flag is seen.
 __device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a, unsigned target,
@@ -309,11 +305,13 @@ __device__ __forceinline__ void signal_ready(unsigned* cnt, uint64_t* bar, int u
 }
 
 // Whole-warp wrappers: lane 0 waits, every lane gets the verdict, and what was published
-// before the flag is visible to every lane afterwards.
-__device__ __forceinline__ bool warp_wait_flag(const Prog& P, Smem* sm, int cls, unsigned target,
-                                               int code) {
+// before the counter's value is visible to every lane afterwards.
+// Class cls complete for `units` units: its counter has reached units * (chunks per unit).
+__device__ __forceinline__ bool warp_wait_class(const Prog& P, const Geo& G, Smem* sm, int cls,
+                                                unsigned units, int code) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = spin_geq(P, sm, my_flag(P, cls), target, code);
+  if ((threadIdx.x & 31) == 0)
+    ok = spin_geq(P, sm, P.s.ctrl + cnt_word(cls), units * (unsigned)G.ncl[cls], code);
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;
@@ -352,34 +350,23 @@ __device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t
 // ------------------------------------------------------------------------------------------
 // Called by the whole warp after the global stores of its last chunk of a run were issued,
 // with `mine` = the number of chunks of the run this warp did. One CTA-scope release-acquire
-// add per warp and run; the warp that completes the CTA's run of (unit, class) orders every
-// warp's stores of the run (CTA-scope acquire, then a gpu-scope fence) before its atomic on
-// the class counter, and the warp whose atomic completes the class for the unit writes the
-// flag of every CTA (release stores).
+// add per warp and run; the warp that completes the CTA's run of (unit, class) has acquired
+// every warp's stores of the run and adds the run's chunks to the class counter with one
+// gpu-scope release-acquire atomic (withheld for the router class under the timeout-test
+// flag, so that the routing decision never comes).
 __device__ __forceinline__ void finish_run(const Prog& P, const Geo& G, Smem* sm, int cls, int u,
                                            unsigned mine) {
-  const int lane = threadIdx.x & 31;
   __syncwarp();
-  int bcast = 0;
-  if (lane == 0) {
+  if ((threadIdx.x & 31) == 0) {
     const unsigned old = atom_add_acq_rel_cta_smem(&sm->run_cnt[cls], mine);
     const unsigned nrun = run_len(G, u, cls);
     if (old + mine == nrun) {
       atom_exch_cta_smem(&sm->run_cnt[cls], 0u);
-      const unsigned og = atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cls), nrun);
-      bcast = og + nrun == (unsigned)(u + 1) * (unsigned)G.ncl[cls];
+      if (!(cls == CL_ROUTER && (P.debug & 1)))
+        atom_add_acq_rel_gpu(P.s.ctrl + cnt_word(cls), nrun);
     }
   }
-  bcast = __shfl_sync(0xffffffffu, bcast, 0);
-  if (bcast && !(cls == CL_ROUTER && (P.debug & 1))) {
-    // One fence per lane (after lane 0's acquire of the counter, through the warp sync), then
-    // relaxed stores: a release store each would wait for the previous one, and the CTAs
-    // served last would see the flag microseconds later.
-    __syncwarp();
-    fence_acq_rel_gpu();
-    for (int c = lane; c < (int)gridDim.x; c += 32)
-      st_relaxed_gpu(P.s.flags + c * F_WORDS + cls, (unsigned)(u + 1));
-  }
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -492,31 +479,20 @@ __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   unsigned i = 0;
   bool failed = false;
   while (i < n_local) {
-    // routing of the first chunk's unit, if it is routed and new
-    {
-      const Chunk c0 = chunk_view(G, cw.u, cw.c);
-      if ((c0.kind == K_RGU || (c0.kind == K_DN && G.routed_on)) && c0.u != rt_u) {
-        int ok = 1;
-        if (lane == 0)
-          ok = wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(c0.u + 1),
-                          DE_TIMEOUT_ROUTE) != 0u;
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-          failed = true;
-          break;
-        }
-        __syncwarp();
-        rt_u = c0.u;
-      }
-    }
-    // deal the lanes out to the copies of the next chunks (the same plan in every lane)
+    // deal the lanes out to the copies of the next chunks (the same plan in every lane); a
+    // step never spans the routing boundary of a unit, and is planned before the wait for
+    // that routing decision, so that the copies go out as soon as it is made
+    const Chunk c0 = chunk_view(G, cw.u, cw.c);
+    const bool wait_rt = (c0.kind == K_RGU || (c0.kind == K_DN && G.routed_on)) && c0.u != rt_u;
+    const int bu = wait_rt ? c0.u : rt_u;  // the unit whose routing this step may use
     Chunk my{};
     int my_q = -1;
     unsigned my_i = 0;
     int nb = 0, used = 0;
     ChunkWalk w = cw;
     while (nb < 8 && i + (unsigned)nb < n_local) {
-      const Chunk c = chunk_view(G, w.u, w.c);
-      if ((c.kind == K_RGU || (c.kind == K_DN && G.routed_on)) && c.u != rt_u) break;
+      const Chunk c = nb == 0 ? c0 : chunk_view(G, w.u, w.c);
+      if ((c.kind == K_RGU || (c.kind == K_DN && G.routed_on)) && c.u != bu) break;
       const int nc = copies_of(G, c);
       if (used + nc > 32) break;
       if (lane >= used && lane < used + nc) {
@@ -527,6 +503,18 @@ __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       used += nc;
       ++nb;
       w.next();
+    }
+    if (wait_rt) {  // the CTA's routing decision of the step's unit
+      int ok = 1;
+      if (lane == 0)
+        ok = wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(c0.u + 1),
+                        DE_TIMEOUT_ROUTE) != 0u;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        failed = true;
+        break;
+      }
+      __syncwarp();
+      rt_u = c0.u;
     }
     // stages free?
     int ok = 1;
@@ -820,7 +808,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     const UnitView uv = unit_view(P, G, u);
     const bool owner = ((unsigned long long)u * ntot) % gridDim.x == blockIdx.x;
     // ---- x(u): needs unit u-1 complete (its output is this input, its buffers are free)
-    if (u > 0 && !warp_wait_flag(P, sm, fcl, (unsigned)u, DE_TIMEOUT_DEP)) break;
+    if (u > 0 && !warp_wait_class(P, G, sm, fcl, (unsigned)u, DE_TIMEOUT_DEP)) break;
     float f = 1.f;
     if (uv.norm) f = rsqrtf(__ldcg(P.s.normsq + (u - 1)) / (float)G.H + P.eps);
     if (!stage_in(P, sm, XA, uv.xin, 4u * (unsigned)G.H, xphase)) break;
@@ -847,7 +835,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     // ---- routing decision: needs every router chunk of unit u
     float sigma = 1.f;
     if (G.route_on) {
-      if (!warp_wait_flag(P, sm, CL_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) break;
+      if (!warp_wait_class(P, G, sm, CL_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) break;
       const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
       if (G.gate_on)  // sigma(g . x): the shared-gate row is router row E
         sigma = (float)(1.0 / (1.0 + exp(-unit_logit(G, lg, G.E))));
@@ -859,7 +847,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     }
     // ---- down input [sigma*h_s | w_0*h_0 | ...]: needs every gate/up chunk of unit u
     if (G.nseg > 0) {
-      if (!warp_wait_flag(P, sm, CL_GU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
+      if (!warp_wait_class(P, G, sm, CL_GU, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
       const unsigned bs = G.shared_on ? 4u * (unsigned)G.I : 0u;
       const unsigned bk = G.routed_on ? 4u * (unsigned)(G.K * G.I) : 0u;
       if (lane == 0) {

@@ -37,13 +37,11 @@ enum Kind { K_ROUTER = 0, K_SGU = 1, K_RGU = 2, K_DN = 3, K_COUNT = 4 };
 enum Class { CL_ROUTER = 0, CL_GU = 1, CL_DN = 2, CL_COUNT = 3 };
 
 // Control words (uint32, zeroed before every launch). Class counters take one atomic per CTA
-// per run of same-class chunks; the CTA whose atomic completes a class for a unit writes
-// "class c of unit u is complete" into every CTA's own flag line, and waiters poll only their
-// own line.
+// per run of same-class chunks; class c is complete for units 0..u when its counter reaches
+// (u + 1) * ncl[c], which the waiters (one warp per CTA) read directly.
 enum Ctrl {
   C_CNT = 0,                    // C_CNT + 32*class: chunks of that class completed (all units)
-  C_WORDS = 32 * CL_COUNT,      // every counter on its own 128-byte line
-  F_WORDS = 32                  // per-CTA flag line: word c = units whose class c is complete
+  C_WORDS = 32 * CL_COUNT       // every counter on its own 128-byte line
 };
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
@@ -94,7 +92,6 @@ struct Geo {
 
 struct Scratch {
   unsigned* ctrl;        // C_WORDS
-  unsigned* flags;       // [gridDim][F_WORDS]
   int* err;              // sticky per-device error word
   double* logits;        // [2][rseg][nr] partial logits per column segment
   float* hs;             // [2][I]
