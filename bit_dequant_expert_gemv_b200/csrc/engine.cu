@@ -835,15 +835,18 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
     // ---- routing decision: needs every router chunk of unit u
     float sigma = 1.f;
     if (G.route_on) {
+      // the unit's logit bias into L2 while the router runs (it streams from HBM otherwise)
+      if (uv.bias)
+        for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
       if (!warp_wait_class(P, G, sm, CL_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) break;
       const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
-      if (G.gate_on)  // sigma(g . x): the shared-gate row is router row E
-        sigma = (float)(1.0 / (1.0 + exp(-unit_logit(G, lg, G.E))));
-      if (lane == 0) sm->sigma[u & 1] = sigma;
       topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
                 owner ? uv.w_out : nullptr);
       __syncwarp();
       if (lane == 0) signal_ready(&sm->rt_ready, &sm->rt_bar, u);
+      // sigma(g . x) (the shared-gate row is router row E) is needed only by the down input
+      if (G.gate_on) sigma = (float)(1.0 / (1.0 + exp(-unit_logit(G, lg, G.E))));
+      if (lane == 0) sm->sigma[u & 1] = sigma;
     }
     // ---- down input [sigma*h_s | w_0*h_0 | ...]: needs every gate/up chunk of unit u
     if (G.nseg > 0) {
