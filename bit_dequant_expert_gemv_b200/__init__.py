@@ -132,7 +132,7 @@ def describe_geometry(H, I, E, K, bits, flags=15, max_smem=232448) -> dict:
     names = ("H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr rseg "
              "rcols rrows nrb R nb nseg Rd n0 n1 n2 n3 off0 off1 off2 off3 off4 ncl0 ncl1 ncl2 "
              "gu_nsl gu_S gu_P gu_nrl dn_nsl dn_S dn_P dn_nrl stage_bytes nstage o_ring o_full "
-             "o_empty o_xa o_sxa o_xg o_sxg o_red o_misc smem_bytes").split()
+             "o_empty o_xa o_xg o_red o_misc smem_bytes").split()
     buf = (C.c_int64 * len(names))()
     n = lib().fmoe_describe_geometry(H, I, E, K, bits, flags, max_smem, buf, len(names))
     if n < 0:

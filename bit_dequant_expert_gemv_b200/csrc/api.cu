@@ -210,10 +210,9 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
     o = align_up(o + bytes, 128);
     return at;
   };
-  G->o_xa = take(4u * (unsigned)std::max(H, G->nseg * I));  // x (raw) / down input (transformed)
-  G->o_sxa = take(4u * (unsigned)std::max(1, G->nseg * I / 32));
-  G->o_xg = take(4u * H);                                     // x transformed
-  G->o_sxg = take(4u * (H / 32));
+  // x (raw) / down input (digit form); x in digit form: 128 bytes per 32-column slice either way
+  G->o_xa = take(4u * (unsigned)std::max(H, G->nseg * I));
+  G->o_xg = take(4u * H);
   G->o_red = take(4u * kConsumerWarps * 16 * kRowsPerLane);   // per-warp row sums
   G->o_misc = take(512);
   const unsigned fixed = o;
@@ -228,7 +227,7 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   // final layout: ring | fixed areas | barriers
   const unsigned ring = (unsigned)ns * G->stage_bytes;
   G->o_ring = 0;
-  G->o_xa += ring; G->o_sxa += ring; G->o_xg += ring; G->o_sxg += ring; G->o_red += ring;
+  G->o_xa += ring; G->o_xg += ring; G->o_red += ring;
   G->o_misc += ring;
   G->o_full = ring + fixed;
   G->o_empty = G->o_full + 8u * ns;
@@ -358,7 +357,7 @@ int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int 
                        G.n[3], G.off[0], G.off[1], G.off[2], G.off[3], G.off[4], G.ncl[0],
                        G.ncl[1], G.ncl[2], G.gu.nsl, G.gu.S, G.gu.P, G.gu.nrl, G.dn.nsl, G.dn.S,
                        G.dn.P, G.dn.nrl, G.stage_bytes, G.nstage, G.o_ring, G.o_full, G.o_empty,
-                       G.o_xa, G.o_sxa, G.o_xg, G.o_sxg, G.o_red, G.o_misc, G.smem_bytes};
+                       G.o_xa, G.o_xg, G.o_red, G.o_misc, G.smem_bytes};
   const int n = (int)(sizeof v / sizeof v[0]);
   for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
   return n < n_out ? n : n_out;

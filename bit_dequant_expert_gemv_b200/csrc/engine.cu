@@ -717,12 +717,65 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
 // the 8 lanes of a quarter-warp reading "float4 i of their own slices" hit distinct banks.
 __device__ __forceinline__ int xpos(int t, int i) { return 32 * t + 4 * (i ^ (t & 7)); }
 
-// x' transform of 4 consecutive values (c a multiple of 4) into the form the slice kernels
-// read: 4-bit pairs (x0, x1/16 - x0); 2-bit quads (x0, x1/4 - x0, x2/16 - x1/4, x3/64 - x2/16).
-__device__ __forceinline__ float4 xform(float4 v, int bits) {
-  if (bits == 4) return make_float4(v.x, v.y * 0.0625f - v.x, v.z, v.w * 0.0625f - v.z);
-  return make_float4(v.x, v.y * 0.25f - v.x, v.z * 0.0625f - v.y * 0.25f,
-                     v.w * 0.015625f - v.z * 0.0625f);
+// Three signed 8-bit digits of r in [-127, 127]: r ~ d0 + d1/128 + d2/16384 with
+// |error| <= 2^-15, each digit rounded to nearest (adding 1.5 * 2^23 leaves the rounded
+// integer in the low mantissa bits; the remainders and their scaling by 128 are exact).
+__device__ __forceinline__ void digits3(float r, int& d0, int& d1, int& d2) {
+  constexpr float kM = 12582912.f;  // 1.5 * 2^23, bit pattern 0x4B400000
+  r = fminf(fmaxf(r, -127.f), 127.f);
+  float t = r + kM;
+  d0 = __float_as_int(t) - 0x4B400000;
+  r = (r - (t - kM)) * 128.f;
+  t = r + kM;
+  d1 = __float_as_int(t) - 0x4B400000;
+  r = (r - (t - kM)) * 128.f;
+  t = r + kM;
+  d2 = __float_as_int(t) - 0x4B400000;
+}
+
+// low bytes of four ints, in order, as one word
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return __byte_perm(__byte_perm((uint32_t)a, (uint32_t)b, 0x0040),
+                     __byte_perm((uint32_t)c, (uint32_t)d, 0x0040), 0x5410);
+}
+
+// Column of byte b of digit word n of a slice, matching the bytes the slice kernels cut from
+// a code word: at 4 bits word n pairs with the low (n even) or high (n odd) nibbles of code
+// word n/2 (columns 8(n/2) + 2b + n%2); at 2 bits with bit-plane n%4 of code word n/4
+// (columns 16(n/4) + 4b + n%4).
+template <int BITS>
+__device__ __forceinline__ constexpr int digit_col(int n, int b) {
+  return BITS == 4 ? 8 * (n >> 1) + 2 * b + (n & 1) : 16 * (n >> 2) + 4 * b + (n & 3);
+}
+
+// The digit form of one 32-value slice v (already scaled): scale s = max|v| / 127 and the
+// digits of v/s, so that v ~ s * (d0 + d1/128 + d2/16384) to within 2.4e-7 * max|v|. Chunk
+// i < 6 of the slice (at xpos(t, i)) holds digit plane i/2, words 4(i%2) .. 4(i%2)+3; chunk 6
+// holds {s, sum of v}.
+template <int BITS>
+__device__ __forceinline__ void store_digits(const float (&v)[32], float* xt, int t) {
+  float m = 0.f, sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) sum += (v[j] + v[j + 1]) + (v[j + 2] + v[j + 3]);
+  const float inv = m > 0.f ? 127.f / m : 0.f;
+  uint32_t w[3][8];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    int d[3][4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) digits3(v[digit_col<BITS>(n, b)] * inv, d[0][b], d[1][b], d[2][b]);
+#pragma unroll
+    for (int p = 0; p < 3; ++p) w[p][n] = pack4(d[p][0], d[p][1], d[p][2], d[p][3]);
+  }
+#pragma unroll
+  for (int i = 0; i < 6; ++i) {
+    const int p = i >> 1, n0 = 4 * (i & 1);
+    *reinterpret_cast<uint4*>(xt + xpos(t, i)) =
+        make_uint4(w[p][n0], w[p][n0 + 1], w[p][n0 + 2], w[p][n0 + 3]);
+  }
+  *reinterpret_cast<float2*>(xt + xpos(t, 6)) = make_float2(m * (1.f / 127.f), sum);
 }
 
 // Bring up to two blocks from global memory (written by other CTAs or by the caller) into
@@ -743,30 +796,26 @@ __device__ __forceinline__ bool stage_in(const Prog& P, Smem* sm, void* dst, con
 }
 
 // Share w (of 8) of a transform: slices [w*nsl/8, (w+1)*nsl/8) of the raw values in `raw`
-// (linear layout) go into `xt` (swizzled) with their sums in `sx`, slice t scaled by
-// scale_of(t) first. One lane per slice (consecutive slices: the swizzle keeps each
-// quarter-warp on distinct banks); raw and xt may be the same array (a lane reads its whole
-// slice before it writes it). Returns the number of slices done.
+// (linear layout), slice t scaled by scale_of(t), go into `xt` in digit form (store_digits).
+// One lane per slice; raw and xt may be the same array (a lane reads its whole slice before
+// it writes it). Returns the number of slices done.
 template <typename ScaleOf>
-__device__ __forceinline__ int transform_share(const float* raw, float* xt, float* sx, int nsl,
-                                               int w, int bits, ScaleOf scale_of) {
+__device__ __forceinline__ int transform_share(const float* raw, float* xt, int nsl, int w,
+                                               int bits, ScaleOf scale_of) {
   const int lane = threadIdx.x & 31;
   const int t0 = w * nsl / 8, t1 = (w + 1) * nsl / 8;
   for (int t = t0 + lane; t < t1; t += 32) {
     const float f = scale_of(t);
-    float4 v[8];
+    float v[32];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // v[i] = logical float4 q = i ^ (t & 7): distinct banks
-      v[i] = *reinterpret_cast<const float4*>(raw + 32 * t + 4 * (i ^ (t & 7)));
-      v[i].x *= f; v[i].y *= f; v[i].z *= f; v[i].w *= f;
+    for (int q = 0; q < 8; ++q) {
+      const float4 a = *reinterpret_cast<const float4*>(raw + 32 * t + 4 * q);
+      v[4 * q] = a.x * f; v[4 * q + 1] = a.y * f; v[4 * q + 2] = a.z * f; v[4 * q + 3] = a.w * f;
     }
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)  // logical q = i ^ (t & 7) belongs at xpos(t, q) = 32t + 4i
-      *reinterpret_cast<float4*>(xt + 32 * t + 4 * i) = xform(v[i], bits);
-    sx[t] = sum;
+    if (bits == 4)
+      store_digits<4>(v, xt, t);
+    else
+      store_digits<2>(v, xt, t);
   }
   __syncwarp();
   return t1 - t0;
@@ -796,9 +845,7 @@ __device__ __forceinline__ float xd_scale(const Geo& G, const Smem* sm, int u, i
 __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   const int lane = threadIdx.x & 31;
   float* XA = reinterpret_cast<float*>(smem + G.o_xa);
-  float* SXA = reinterpret_cast<float*>(smem + G.o_sxa);
   float* XG = reinterpret_cast<float*>(smem + G.o_xg);
-  float* SXG = reinterpret_cast<float*>(smem + G.o_sxg);
   const int fcl = final_class(G);
   const unsigned ntot = (unsigned)G.off[K_COUNT];
   const bool gu_on = G.shared_on || G.routed_on;
@@ -829,7 +876,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       int done = 0;
       for (int w = 0; w < kConsumerWarps; ++w)
         if (!warp_in_range(lo, hi, w))
-          done += transform_share(XA, XG, SXG, G.H / 32, w, G.bits, [&](int) { return f; });
+          done += transform_share(XA, XG, G.H / 32, w, G.bits, [&](int) { return f; });
       if (done && lane == 0) red_release_cta_smem(&sm->xg_done[u & 1], (unsigned)done);
     }
     // ---- routing decision: needs every router chunk of unit u
@@ -868,7 +915,7 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       int done = 0;
       for (int w = 0; w < kConsumerWarps; ++w)
         if (!warp_in_range(lo, hi, w))
-          done += transform_share(XA, XA, SXA, G.nseg * (G.I / 32), w, G.bits,
+          done += transform_share(XA, XA, G.nseg * (G.I / 32), w, G.bits,
                                   [&](int t) { return xd_scale(G, sm, u, t); });
       if (done && lane == 0) red_release_cta_smem(&sm->xd_done[u & 1], (unsigned)done);
     }
@@ -878,19 +925,15 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
 // ------------------------------------------------------------------------------------------
 // dequantising dot products: W rows x one 32-column slice
 // ------------------------------------------------------------------------------------------
-// One byte of codes becomes the binary32 32768 + byte (exponent 15, byte in mantissa bits
-// 8..15); clearing the low code(s) gives 32768 + the high part. Subtracting 32768 is exact.
-__device__ __forceinline__ uint32_t magic_byte(uint32_t word, int k) {
-  return __byte_perm(word, 0x47000000u, 0x7604u | ((uint32_t)k << 4));
-}
-
 // acc[w] += s_w * sum(q x) + z_w * sum(x) over the slice, for W rows whose codes start at
 // stage + coff[w] and whose scale/bias word is at stage + soff[w]; rows with ok[w] false add
-// 0 (their offsets must still point inside the stage). xq: the slice's transformed x.
+// 0 (their offsets must still point inside the stage). sum(q x) comes from integer dot
+// products of the codes with the slice's three digit planes xd (store_digits), scaled by sc;
+// sx is sum(x).
 template <int BITS, int W>
 __device__ __forceinline__ void qslice(uint32_t stage, const unsigned (&coff)[W],
                                        const unsigned (&soff)[W], const bool (&ok)[W],
-                                       const float (&xq)[32], float sx, float* acc) {
+                                       const int (&xd)[24], float sc, float sx, float* acc) {
   constexpr int kWords = BITS == 4 ? 4 : 2;
   uint32_t q[W][kWords];
   uint32_t sbw[W];
@@ -905,44 +948,26 @@ __device__ __forceinline__ void qslice(uint32_t stage, const unsigned (&coff)[W]
     }
     sbw[w] = lds32(stage + soff[w]);
   }
-  const float2 m = make_float2(-32768.f, -32768.f);
-  float2 a0[W], a1[W];
+  int c0[W], c1[W], c2[W];
 #pragma unroll
-  for (int w = 0; w < W; ++w) {
-    a0[w] = make_float2(0.f, 0.f);
-    a1[w] = make_float2(0.f, 0.f);
-  }
+  for (int w = 0; w < W; ++w) c0[w] = c1[w] = c2[w] = 0;
 #pragma unroll
   for (int wi = 0; wi < kWords; ++wi) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int b = wi * 4 + k;
-      if constexpr (BITS == 4) {
-        // (16*hi + lo, 16*hi) paired with (x_lo, x_hi/16 - x_lo)
-        const float2 xv = make_float2(xq[2 * b], xq[2 * b + 1]);
+    for (int w = 0; w < W; ++w) {
+      if constexpr (BITS == 4) {  // low nibbles: digit word 2wi, high nibbles: 2wi + 1
+        const int lo = (int)(q[w][wi] & 0x0F0F0F0Fu);
+        const int hi = (int)((q[w][wi] >> 4) & 0x0F0F0F0Fu);
+        c0[w] = __dp4a(hi, xd[2 * wi + 1], __dp4a(lo, xd[2 * wi], c0[w]));
+        c1[w] = __dp4a(hi, xd[8 + 2 * wi + 1], __dp4a(lo, xd[8 + 2 * wi], c1[w]));
+        c2[w] = __dp4a(hi, xd[16 + 2 * wi + 1], __dp4a(lo, xd[16 + 2 * wi], c2[w]));
+      } else {  // bit-plane p of code word wi: digit word 4wi + p
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          const uint32_t t = magic_byte(q[w][wi], k);
-          const float2 f =
-              __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFF0FFu)), m);
-          if (b & 1)
-            a1[w] = __ffma2_rn(f, xv, a1[w]);
-          else
-            a0[w] = __ffma2_rn(f, xv, a0[w]);
-        }
-      } else {
-        // (c0+4c1+16c2+64c3, 4c1+16c2+64c3) and (16c2+64c3, 64c3)
-        const float2 xa = make_float2(xq[4 * b], xq[4 * b + 1]);
-        const float2 xb = make_float2(xq[4 * b + 2], xq[4 * b + 3]);
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-          const uint32_t t = magic_byte(q[w][wi], k);
-          const float2 f01 =
-              __fadd2_rn(make_float2(__uint_as_float(t), __uint_as_float(t & 0xFFFFFCFFu)), m);
-          const float2 f23 = __fadd2_rn(
-              make_float2(__uint_as_float(t & 0xFFFFF0FFu), __uint_as_float(t & 0xFFFFC0FFu)), m);
-          a0[w] = __ffma2_rn(f01, xa, a0[w]);
-          a1[w] = __ffma2_rn(f23, xb, a1[w]);
+        for (int p = 0; p < 4; ++p) {
+          const int c = (int)((q[w][wi] >> (2 * p)) & 0x03030303u);
+          c0[w] = __dp4a(c, xd[4 * wi + p], c0[w]);
+          c1[w] = __dp4a(c, xd[8 + 4 * wi + p], c1[w]);
+          c2[w] = __dp4a(c, xd[16 + 4 * wi + p], c2[w]);
         }
       }
     }
@@ -951,7 +976,8 @@ __device__ __forceinline__ void qslice(uint32_t stage, const unsigned (&coff)[W]
   for (int w = 0; w < W; ++w) {
     const float s = __uint_as_float(sbw[w] << 16);
     const float z = __uint_as_float(sbw[w] & 0xFFFF0000u);
-    const float qx = (a0[w].x + a0[w].y) + (a1[w].x + a1[w].y);
+    const float qx =
+        sc * ((float)c0[w] + ((float)c1[w] * 0.0078125f + (float)c2[w] * 6.103515625e-05f));
     acc[w] += ok[w] ? fmaf(s, qx, z * sx) : 0.f;
   }
 }
@@ -1005,7 +1031,7 @@ struct RowGeom {
 // red[(rho % P) * kRowsPerLane + rho / P].
 template <int BITS, int NRL, typename Valid>
 __device__ __forceinline__ void dot_chunk(uint32_t st, const LaneMap& M, const RowGeom& RG,
-                                          int nrows, Valid valid, uint32_t xs, uint32_t sxs,
+                                          int nrows, Valid valid, uint32_t xs,
                                           float* red) {
   constexpr int NRLP = NRL <= 4 ? 4 : 8;         // padded to a power of two for the butterfly
   constexpr int GW = (NRL % 4 == 0) ? 4 : 3;     // rows per lock-step group
@@ -1020,14 +1046,15 @@ __device__ __forceinline__ void dot_chunk(uint32_t st, const LaneMap& M, const R
     const int t = lane_s + M.S * j;
     const bool tok = t < M.nsl;
     const int tc = tok ? t : M.nsl - 1;
-    float xq[32];
+    int xd[24];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 6; ++i) {
       const uint4 a = lds128(xs + 4u * (unsigned)xpos(tc, i));
-      xq[4 * i] = __uint_as_float(a.x); xq[4 * i + 1] = __uint_as_float(a.y);
-      xq[4 * i + 2] = __uint_as_float(a.z); xq[4 * i + 3] = __uint_as_float(a.w);
+      xd[4 * i] = (int)a.x; xd[4 * i + 1] = (int)a.y; xd[4 * i + 2] = (int)a.z;
+      xd[4 * i + 3] = (int)a.w;
     }
-    const float sx = __uint_as_float(lds32(sxs + 4u * (unsigned)tc));
+    const uint2 ss = lds64(xs + 4u * (unsigned)xpos(tc, 6));
+    const float sc = __uint_as_float(ss.x), sx = __uint_as_float(ss.y);
     const int seg = tc / RG.spseg, loc = tc - seg * RG.spseg;
     const unsigned cbase = (unsigned)seg * RG.seg_c + (unsigned)loc * cb;
     const unsigned sbase = RG.sb0 + (unsigned)seg * RG.seg_s + (unsigned)(loc >> 1) * 4u;
@@ -1044,7 +1071,7 @@ __device__ __forceinline__ void dot_chunk(uint32_t st, const LaneMap& M, const R
           coff[w] = cbase + rr * RG.rc;
           soff[w] = sbase + rr * RG.rs;
         }
-        qslice<BITS, GW>(st, coff, soff, ok, xq, sx, acc + g);
+        qslice<BITS, GW>(st, coff, soff, ok, xd, sc, sx, acc + g);
       }
     }
   }
@@ -1099,7 +1126,7 @@ __device__ __forceinline__ void router_chunk(const Prog& P, const Geo& G, const 
 template <int BITS, int NRL>
 __device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, const Chunk& cv,
                                          const uint8_t* stage, uint64_t* empty, const float* XG,
-                                         const float* SXG, float* red) {
+                                         float* red) {
   const int lane = threadIdx.x & 31;
   RowGeom RG;
   RG.rc = G.rc_h; RG.rs = G.rs_h; RG.seg_c = 0; RG.seg_s = 0;
@@ -1109,7 +1136,7 @@ __device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, const Chun
   dot_chunk<BITS, NRL>(
       smem_u32(stage), G.gu, RG, 2 * R,
       [&](int rho) { return rho < 2 * R && (rho < R ? rho : rho - R) < n; }, smem_u32(XG),
-      smem_u32(SXG), red);
+      red);
   release_stage(empty);
   __syncwarp();
   float* h = cv.kind == K_SGU ? P.s.hs + (size_t)(cv.u & 1) * G.I
@@ -1125,7 +1152,7 @@ __device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, const Chun
 template <int BITS, int NRL>
 __device__ __forceinline__ void dn_chunk(const Prog& P, const Geo& G, const Chunk& cv,
                                          const UnitView& uv, const uint8_t* stage,
-                                         uint64_t* empty, const float* XD, const float* SXD,
+                                         uint64_t* empty, const float* XD,
                                          float* red) {
   const int lane = threadIdx.x & 31;
   // the residual each output row adds is fetched first so its latency hides behind the dots
@@ -1138,7 +1165,7 @@ __device__ __forceinline__ void dn_chunk(const Prog& P, const Geo& G, const Chun
   RG.spseg = G.I / 32;
   const int n = cv.n;
   dot_chunk<BITS, NRL>(smem_u32(stage), G.dn, RG, n, [&](int rho) { return rho < n; },
-                       smem_u32(XD), smem_u32(SXD), red);
+                       smem_u32(XD), red);
   release_stage(empty);
   __syncwarp();
   float sq = 0.f;
@@ -1167,21 +1194,19 @@ __device__ __forceinline__ void dispatch_dot(const Prog& P, const Geo& G, const 
                                              uint64_t* empty, uint8_t* smem, float* red) {
   if (cv.kind == K_DN) {
     const float* XD = reinterpret_cast<const float*>(smem + G.o_xa);
-    const float* SXD = reinterpret_cast<const float*>(smem + G.o_sxa);
     switch (nrl_class(G.dn.nrl)) {
-      case 3: dn_chunk<BITS, 3>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
-      case 4: dn_chunk<BITS, 4>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
-      case 6: dn_chunk<BITS, 6>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
-      default: dn_chunk<BITS, 8>(P, G, cv, uv, stage, empty, XD, SXD, red); break;
+      case 3: dn_chunk<BITS, 3>(P, G, cv, uv, stage, empty, XD, red); break;
+      case 4: dn_chunk<BITS, 4>(P, G, cv, uv, stage, empty, XD, red); break;
+      case 6: dn_chunk<BITS, 6>(P, G, cv, uv, stage, empty, XD, red); break;
+      default: dn_chunk<BITS, 8>(P, G, cv, uv, stage, empty, XD, red); break;
     }
   } else {
     const float* XG = reinterpret_cast<const float*>(smem + G.o_xg);
-    const float* SXG = reinterpret_cast<const float*>(smem + G.o_sxg);
     switch (nrl_class(G.gu.nrl)) {
-      case 3: gu_chunk<BITS, 3>(P, G, cv, stage, empty, XG, SXG, red); break;
-      case 4: gu_chunk<BITS, 4>(P, G, cv, stage, empty, XG, SXG, red); break;
-      case 6: gu_chunk<BITS, 6>(P, G, cv, stage, empty, XG, SXG, red); break;
-      default: gu_chunk<BITS, 8>(P, G, cv, stage, empty, XG, SXG, red); break;
+      case 3: gu_chunk<BITS, 3>(P, G, cv, stage, empty, XG, red); break;
+      case 4: gu_chunk<BITS, 4>(P, G, cv, stage, empty, XG, red); break;
+      case 6: gu_chunk<BITS, 6>(P, G, cv, stage, empty, XG, red); break;
+      default: gu_chunk<BITS, 8>(P, G, cv, stage, empty, XG, red); break;
     }
   }
 }
@@ -1191,9 +1216,7 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + G.o_empty);
   float* red = reinterpret_cast<float*>(smem + G.o_red) + (size_t)w * 16 * kRowsPerLane;
   float* XA = reinterpret_cast<float*>(smem + G.o_xa);
-  float* SXA = reinterpret_cast<float*>(smem + G.o_sxa);
   float* XG = reinterpret_cast<float*>(smem + G.o_xg);
-  float* SXG = reinterpret_cast<float*>(smem + G.o_sxg);
   const int lane = threadIdx.x & 31;
   const unsigned NS = (unsigned)G.nstage;
   const unsigned n_local = local_chunks(P, G);
@@ -1224,7 +1247,7 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
       if (xd_mine != need) {
         xd_mine = need;
         share_wait = true;
-        const int d = transform_share(XA, XA, SXA, G.nseg * (G.I / 32), w, G.bits,
+        const int d = transform_share(XA, XA, G.nseg * (G.I / 32), w, G.bits,
                                       [&](int t) { return xd_scale(G, sm, cv.u, t); });
         if (lane == 0 && d) red_release_cta_smem(&sm->xd_done[cv.u & 1], (unsigned)d);
       }
@@ -1237,7 +1260,7 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
         xg_mine = need;
         share_wait = true;
         const float f = sm->xf[cv.u & 1];
-        const int d = transform_share(XA, XG, SXG, G.H / 32, w, G.bits,
+        const int d = transform_share(XA, XG, G.H / 32, w, G.bits,
                                       [&](int) { return f; });
         if (lane == 0 && d) red_release_cta_smem(&sm->xg_done[cv.u & 1], (unsigned)d);
       }

@@ -86,7 +86,7 @@ struct Geo {
   // shared memory carve-up (byte offsets from the dynamic smem base)
   unsigned stage_bytes;
   int nstage;
-  unsigned o_ring, o_full, o_empty, o_xa, o_sxa, o_xg, o_sxg, o_red, o_misc;
+  unsigned o_ring, o_full, o_empty, o_xa, o_xg, o_red, o_misc;
   unsigned smem_bytes;
 };
 

@@ -135,16 +135,15 @@ def test_geometry_in_bounds(shape, flags):
     nseg = G["nseg"]
     xa_len = 4 * max(H, nseg * I)
     # carve-up: ring | fixed areas | barriers, non-overlapping and in order
-    areas = [("ring", 0, ns * sb), ("xa", G["o_xa"], xa_len),
-             ("sxa", G["o_sxa"], 4 * max(1, nseg * I // 32)), ("xg", G["o_xg"], 4 * H),
-             ("sxg", G["o_sxg"], 4 * (H // 32)),
+    # x areas: 128 bytes per 32-column slice (raw floats, or six digit chunks + {scale, sum})
+    areas = [("ring", 0, ns * sb), ("xa", G["o_xa"], xa_len), ("xg", G["o_xg"], 4 * H),
              ("red", G["o_red"], 4 * CONSUMER_WARPS * 16 * ROWS_PER_LANE),
              ("misc", G["o_misc"], 512), ("full", G["o_full"], 8 * ns), ("empty", G["o_empty"], 8 * ns)]
     for (n1, a1, l1), (n2, a2, l2) in zip(areas, areas[1:]):
         assert a1 + l1 <= a2, (n1, n2)
     assert areas[-1][1] + areas[-1][2] <= G["smem_bytes"]
     assert G["o_full"] % 8 == 0 and G["o_misc"] % 16 == 0
-    for name in ("o_xa", "o_sxa", "o_xg", "o_sxg", "o_red"):
+    for name in ("o_xa", "o_xg", "o_red"):
         assert G[name] % 16 == 0, name
     # stager bulk copies into XA: x, then h_s | h_k
     assert 4 * H <= xa_len and 4 * (nseg * I) <= xa_len
