@@ -479,42 +479,65 @@ __device__ void producer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   unsigned i = 0;
   bool failed = false;
   while (i < n_local) {
-    // deal the lanes out to the copies of the next chunks (the same plan in every lane); a
-    // step never spans the routing boundary of a unit, and is planned before the wait for
-    // that routing decision, so that the copies go out as soon as it is made
-    const Chunk c0 = chunk_view(G, cw.u, cw.c);
-    const bool wait_rt = (c0.kind == K_RGU || (c0.kind == K_DN && G.routed_on)) && c0.u != rt_u;
-    const int bu = wait_rt ? c0.u : rt_u;  // the unit whose routing this step may use
-    Chunk my{};
-    int my_q = -1;
-    unsigned my_i = 0;
-    int nb = 0, used = 0;
-    ChunkWalk w = cw;
-    while (nb < 8 && i + (unsigned)nb < n_local) {
-      const Chunk c = nb == 0 ? c0 : chunk_view(G, w.u, w.c);
-      if ((c.kind == K_RGU || (c.kind == K_DN && G.routed_on)) && c.u != bu) break;
-      const int nc = copies_of(G, c);
-      if (used + nc > 32) break;
-      if (lane >= used && lane < used + nc) {
-        my = c;
-        my_q = lane - used;
-        my_i = i + (unsigned)nb;
-      }
-      used += nc;
-      ++nb;
-      w.next();
+    // Plan a step (the same plan in every lane): lane j <= 8 decodes the step's chunk j (the
+    // walk advanced j chunks), a warp scan of the chunks' copy counts takes the leading
+    // chunks that fit 32 copies (at most 8, never across the routing boundary of a unit), and
+    // each lane picks up its copy. Planned before the wait for that routing decision, so that
+    // the copies go out as soon as it is made.
+    ChunkWalk wj = cw;
+    const int jl = lane < 8 ? lane : 8;
+    wj.c += jl * wj.step;
+    while (wj.c >= wj.ntot) {
+      wj.c -= wj.ntot;
+      ++wj.u;
     }
+    const Chunk cj = chunk_view(G, wj.u, wj.c);
+    const int c0_u = __shfl_sync(0xffffffffu, cj.u, 0);
+    const int c0_kind = __shfl_sync(0xffffffffu, cj.kind, 0);
+    const bool wait_rt =
+        (c0_kind == K_RGU || (c0_kind == K_DN && G.routed_on)) && c0_u != rt_u;
+    const int bu = wait_rt ? c0_u : rt_u;  // the unit whose routing this step may use
+    const bool ok_j = lane < 8 && i + (unsigned)lane < n_local &&
+                      !((cj.kind == K_RGU || (cj.kind == K_DN && G.routed_on)) && cj.u != bu);
+    const int nc_j = ok_j ? copies_of(G, cj) : 0;
+    int incl = nc_j;  // inclusive prefix sum of the copy counts over lanes 0..lane
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const unsigned take = __ballot_sync(0xffffffffu, ok_j && incl <= 32);
+    const int nb = __ffs(~take) - 1;  // leading chunks taken (chunk 0 always fits)
+    int my_j = 0, my_lo = 0;
+    for (int j = 0; j < 8; ++j) {
+      const int ij = __shfl_sync(0xffffffffu, incl, j);
+      if (j < nb && lane >= ij) my_j = j + 1, my_lo = ij;
+    }
+    const int my_q = my_j < nb ? lane - my_lo : -1;
+    const unsigned my_i = i + (unsigned)my_j;
+    Chunk my;
+    my.u = __shfl_sync(0xffffffffu, cj.u, my_j);
+    my.c = __shfl_sync(0xffffffffu, cj.c, my_j);
+    my.kind = __shfl_sync(0xffffffffu, cj.kind, my_j);
+    my.j = __shfl_sync(0xffffffffu, cj.j, my_j);
+    my.r0 = __shfl_sync(0xffffffffu, cj.r0, my_j);
+    my.n = __shfl_sync(0xffffffffu, cj.n, my_j);
+    my.k = __shfl_sync(0xffffffffu, cj.k, my_j);
+    my.seg = __shfl_sync(0xffffffffu, cj.seg, my_j);
+    ChunkWalk w = cw;  // the walk after the step's nb chunks (lane nb decoded it)
+    w.u = __shfl_sync(0xffffffffu, wj.u, nb);
+    w.c = __shfl_sync(0xffffffffu, wj.c, nb);
     if (wait_rt) {  // the CTA's routing decision of the step's unit
       int ok = 1;
       if (lane == 0)
-        ok = wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(c0.u + 1),
+        ok = wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(c0_u + 1),
                         DE_TIMEOUT_ROUTE) != 0u;
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         failed = true;
         break;
       }
       __syncwarp();
-      rt_u = c0.u;
+      rt_u = c0_u;
     }
     // stages free?
     int ok = 1;
@@ -717,20 +740,15 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
 // the 8 lanes of a quarter-warp reading "float4 i of their own slices" hit distinct banks.
 __device__ __forceinline__ int xpos(int t, int i) { return 32 * t + 4 * (i ^ (t & 7)); }
 
-// Three signed 8-bit digits of r in [-127, 127]: r ~ d0 + d1/128 + d2/16384 with
-// |error| <= 2^-15, each digit rounded to nearest (adding 1.5 * 2^23 leaves the rounded
-// integer in the low mantissa bits; the remainders and their scaling by 128 are exact).
-__device__ __forceinline__ void digits3(float r, int& d0, int& d1, int& d2) {
-  constexpr float kM = 12582912.f;  // 1.5 * 2^23, bit pattern 0x4B400000
-  r = fminf(fmaxf(r, -127.f), 127.f);
-  float t = r + kM;
-  d0 = __float_as_int(t) - 0x4B400000;
-  r = (r - (t - kM)) * 128.f;
-  t = r + kM;
-  d1 = __float_as_int(t) - 0x4B400000;
-  r = (r - (t - kM)) * 128.f;
-  t = r + kM;
-  d2 = __float_as_int(t) - 0x4B400000;
+// Three signed 8-bit digits of q = rint(v * k) (|q| <= 127 * 2^14): q = d0 * 2^14 + d1 * 2^7
+// + d2 with d0 in [-127, 127], d1 in [-64, 64], d2 in [-64, 63]. Adding 1.5 * 2^23 in the same
+// fused operation leaves the rounded product in the low mantissa bits.
+__device__ __forceinline__ void digits3(float v, float k, int& d0, int& d1, int& d2) {
+  const int q = __float_as_int(fmaf(v, k, 12582912.f)) - 0x4B400000;
+  d0 = (q + 8192) >> 14;
+  const int r = q - (d0 << 14);
+  d1 = (r + 64) >> 7;
+  d2 = r - (d1 << 7);
 }
 
 // low bytes of four ints, in order, as one word
@@ -759,13 +777,13 @@ __device__ __forceinline__ void store_digits(const float (&v)[32], float* xt, in
   for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
 #pragma unroll
   for (int j = 0; j < 32; j += 4) sum += (v[j] + v[j + 1]) + (v[j + 2] + v[j + 3]);
-  const float inv = m > 0.f ? 127.f / m : 0.f;
+  const float k = m > 0.f ? 2080768.f / m : 0.f;  // 127 * 2^14 / max|v|
   uint32_t w[3][8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) {
     int d[3][4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) digits3(v[digit_col<BITS>(n, b)] * inv, d[0][b], d[1][b], d[2][b]);
+    for (int b = 0; b < 4; ++b) digits3(v[digit_col<BITS>(n, b)], k, d[0][b], d[1][b], d[2][b]);
 #pragma unroll
     for (int p = 0; p < 3; ++p) w[p][n] = pack4(d[p][0], d[p][1], d[p][2], d[p][3]);
   }
