@@ -13,20 +13,21 @@
 //   s * sum(q*x) + z * sum(x) per 32-column slice: the pages' fma(nibble, scale*x, bias*x)
 //   with the scale and bias factored out of the slice sum (same value in real arithmetic;
 //     "Qu'est-ce que Flash-MoE ?" (a2a-mcp.org, fr), §2 "Noyaux de Déquantification Optimisés
-//      pour FMA").
+//      pour FMA"); sum(q*x) is taken as integer dot products of the codes with three 8-bit
+//   digit planes of x (x ~ s_x (d0 + d1/128 + d2/16384), within 3.5e-7 of the slice's largest
+//   |x|), so that one dp4a covers four weights.
 //
 // How: one CTA per SM, every CTA working through a static share of every unit's chunks.
 //   producer warp   streams each chunk's weight rows into a ring of shared-memory stages with
 //                   1-D TMA bulk copies that complete on the stage's mbarrier;
-//   stager warp     per unit: brings x into shared memory (TMA) and prepares its two forms
-//                   (raw for the router, pair-transformed + slice sums for the codes), selects
-//                   the top-K experts once the router is complete, and prepares the down
-//                   input [sigma*h_s | w_k*h_k] once every gate/up chunk is complete;
-//   consumer warps  each owns whole chunks (local chunk i -> warp i mod kConsumerWarps):
-//                   unpacks codes with one byte-permute per byte into a binary32
-//                   "32768 + byte" pattern, finishes the exact code values with packed f32x2
-//                   arithmetic, reduces its row sums inside the warp and runs the chunk's
-//                   epilogue (logit store, SwiGLU, or residual + combine) itself -- no
+//   stager warp     per unit: brings x into shared memory (TMA; the raw copy is the router's
+//                   input), selects the top-K experts once the router is complete, and brings
+//                   in the down input [h_s | h_k] once every gate/up chunk is complete;
+//   consumer warps  each owns whole chunks (local chunk i -> warp i mod kConsumerWarps); each
+//                   puts one eighth of the unit's x and of its down input [sigma*h_s | w_k*h_k]
+//                   into digit form; cuts codes into bytes (nibbles or bit-planes) for dp4a
+//                   against the digit planes, reduces its row sums inside the warp and runs the
+//                   chunk's epilogue (logit store, SwiGLU, or residual + combine) itself -- no
 //                   block-wide barrier and no cross-warp reduction on the hot path.
 // Completion is counted per run of same-class chunks of a CTA: the warp finishing a CTA's run
 // makes one gpu-scope release-acquire atomic on the class counter, and the stager warps poll
