@@ -634,12 +634,97 @@ __device__ __forceinline__ double unit_logit(const Geo& G, const double* lg, int
   return a;
 }
 
-// Top-K of the unit's logits by one warp. Every lane sorts its 16 packed keys; passes over
-// more than 512 experts keep each lane's best 16 by a bitonic merge. Then K rounds of a warp
-// maximum over the lanes' heads (two 32-bit reductions), the winning lane dropping its head.
+// Order-preserving 32-bit key of a binary32 value (larger value <=> larger signed key).
+__device__ __forceinline__ int fkey(float f) {
+  const int b = __float_as_int(f);
+  return b >= 0 ? b : b ^ 0x7FFFFFFF;
+}
+
+// Top-K over at most 512 experts by one warp (lane l holds experts l + 32 i). K rounds: the
+// warp maximum of the lanes' best 32-bit keys (the logit rounded to binary32), then the lowest
+// expert index holding it, so that ties go to the lower index; logits that differ by less than
+// binary32 resolution (~6e-8 relative, far inside the tie band of the routing decision) count
+// as tied. The winners' binary64 logits are carried along for the weights
 // w_k = exp(l_k - l_max) / sum_sel exp(l_j - l_max): the softmax over all experts followed by
-// renormalisation over the selected ones, where the full softmax denominator cancels; the
-// logits come back from the keys with 40 significant bits.
+// renormalisation over the selected ones, where the full softmax denominator cancels.
+__device__ void topk_warp_512(const Geo& G, const double* lg, const float* bias, int* rt_e,
+                              float* rt_w, int* idx_out, float* w_out) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = 16;
+  double lv[kPer], p1[kPer];
+  float bv[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {  // the bias and the first two segments in one round trip
+    const int ec = min(lane + 32 * i, G.E - 1);
+    bv[i] = bias ? __ldcg(bias + ec) : 0.f;
+    lv[i] = __ldcg(lg + ec);
+    p1[i] = G.rseg > 1 ? __ldcg(lg + (size_t)G.nr + ec) : 0.0;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) lv[i] = ((double)bv[i] + lv[i]) + p1[i];
+  for (int sg = 2; sg < G.rseg; ++sg) {
+    double part[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      part[i] = __ldcg(lg + (size_t)sg * G.nr + min(lane + 32 * i, G.E - 1));
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) lv[i] += part[i];
+  }
+  int key[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) key[i] = lane + 32 * i < G.E ? fkey((float)lv[i]) : INT_MIN;
+  // the lane's best: largest key, lowest index on ties
+  auto lane_best = [&](int& bk, int& bi) {
+    bk = key[0];
+    bi = 0;
+#pragma unroll
+    for (int i = 1; i < kPer; ++i)
+      if (key[i] > bk) bk = key[i], bi = i;
+  };
+  int bk, bi;
+  lane_best(bk, bi);
+  int sel_e = 0;
+  double sel_l = 0.0;
+  for (int k = 0; k < G.K; ++k) {
+    const int mk = __reduce_max_sync(0xffffffffu, bk);
+    const int we = (int)__reduce_min_sync(0xffffffffu, bk == mk ? (unsigned)(lane + 32 * bi) : 0xFFFFFFFFu);
+    const bool win = lane == (we & 31);
+    double wl = 0.0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) wl = (win && i == bi) ? lv[i] : wl;
+    wl = __shfl_sync(0xffffffffu, wl, we & 31);
+    if (win) {
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) key[i] = i == bi ? INT_MIN : key[i];
+      lane_best(bk, bi);
+    }
+    if (lane == k) {
+      sel_e = we;
+      sel_l = wl;
+    }
+  }
+  const double l0 = __shfl_sync(0xffffffffu, sel_l, 0);
+  const bool mine = lane < G.K;
+  const float ex = mine ? expf((float)(sel_l - l0)) : 0.f;
+  float den = ex;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (mine) {
+    const int e = min(max(sel_e, 0), G.E - 1);  // NaN logits must not make an address
+    const float wk = __fdividef(ex, den);
+    rt_e[lane] = e;
+    rt_w[lane] = wk;
+    if (idx_out) idx_out[lane] = e;
+    if (w_out) w_out[lane] = wk;
+  }
+  __syncwarp();
+}
+
+// Top-K of the unit's logits by one warp for more than 512 experts. Every lane sorts its 16
+// packed keys; passes over 512 experts at a time keep each lane's best 16 by a bitonic merge.
+// Then K rounds of a warp maximum over the lanes' heads (two 32-bit reductions), the winning
+// lane dropping its head. The weights as in topk_warp_512; the logits come back from the keys
+// with 40 significant bits.
 __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int* rt_e,
                           float* rt_w, int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
@@ -906,8 +991,12 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
         for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
       if (!warp_wait_class(P, G, sm, CL_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) break;
       const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
-      topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
-                owner ? uv.w_out : nullptr);
+      if (G.E <= 512)
+        topk_warp_512(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1],
+                      owner ? uv.idx_out : nullptr, owner ? uv.w_out : nullptr);
+      else
+        topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
+                  owner ? uv.w_out : nullptr);
       __syncwarp();
       if (lane == 0) signal_ready(&sm->rt_ready, &sm->rt_bar, u);
       // sigma(g . x) (the shared-gate row is router row E) is needed only by the down input
