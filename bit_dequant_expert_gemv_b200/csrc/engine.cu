@@ -202,6 +202,9 @@ struct Smem {  // small shared state (in the misc area)
   // consumer warps: one eighth each (the stager does the eighths of warps that have no chunk
   // needing them); per unit parity, the number of slices transformed so far.
   unsigned xg_done[2], xd_done[2];
+  // per unit parity: the warps holding the unit's gate/up (down) chunks share its x (down
+  // input) transform; the first of them (local chunk index mod 8) and how many chunks there are
+  int xg_w0[2], xg_n[2], xd_w0[2], xd_n[2];
   float xf[2];                 // RMSNorm factor of the unit's x (1 without a norm)
   float sigma[2];              // sigmoid(g . x) of the unit (1 without a shared gate)
   volatile int abort;
@@ -899,15 +902,15 @@ __device__ __forceinline__ bool stage_in(const Prog& P, Smem* sm, void* dst, con
   return ok;
 }
 
-// Share w (of 8) of a transform: slices [w*nsl/8, (w+1)*nsl/8) of the raw values in `raw`
+// Share r (of ns) of a transform: slices [r*nsl/ns, (r+1)*nsl/ns) of the raw values in `raw`
 // (linear layout), slice t scaled by scale_of(t), go into `xt` in digit form (store_digits).
 // One lane per slice; raw and xt may be the same array (a lane reads its whole slice before
 // it writes it). Returns the number of slices done.
 template <typename ScaleOf>
-__device__ __forceinline__ int transform_share(const float* raw, float* xt, int nsl, int w,
-                                               int bits, ScaleOf scale_of) {
+__device__ __forceinline__ int transform_share(const float* raw, float* xt, int nsl, int r,
+                                               int ns, int bits, ScaleOf scale_of) {
   const int lane = threadIdx.x & 31;
-  const int t0 = w * nsl / 8, t1 = (w + 1) * nsl / 8;
+  const int t0 = r * nsl / ns, t1 = (r + 1) * nsl / ns;
   for (int t = t0 + lane; t < t1; t += 32) {
     const float f = scale_of(t);
     float v[32];
@@ -933,11 +936,11 @@ __device__ __forceinline__ void local_range(const Geo& G, int u, int c0, int c1,
   *hi = *lo + count_cong(base + (unsigned)c0, base + (unsigned)c1, blockIdx.x, gridDim.x);
 }
 
-// Does consumer warp w get a chunk with local index in [lo, hi)? (local chunk i -> warp i mod 8)
-__device__ __forceinline__ bool warp_in_range(unsigned lo, unsigned hi, int w) {
-  const unsigned cnt = hi - lo;
-  return cnt >= (unsigned)kConsumerWarps ||
-         ((unsigned)(w - (int)(lo % kConsumerWarps) + kConsumerWarps) % kConsumerWarps) < cnt;
+// The share of consumer warp w among the n_sh warps that hold a range of n chunks whose first
+// local chunk goes to warp w0 (local chunk i -> warp i mod 8); the caller holds one of them.
+__device__ __forceinline__ int share_rank(int w0, int n, int w, int* n_sh) {
+  *n_sh = n < kConsumerWarps ? n : kConsumerWarps;
+  return n < kConsumerWarps ? (w - w0 + kConsumerWarps) % kConsumerWarps : w;
 }
 
 // The scale of down-input slice t: sigma for the shared expert's segment, w_k for routed k.
@@ -967,22 +970,18 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       for (int c = lane * 4; c < G.H; c += 128)
         *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XA + c);
     if (lane == 0) {
+      unsigned lo, hi;
       sm->xf[u & 1] = f;
       sm->xg_done[u & 1] = 0u;
+      local_range(G, u, G.off[K_SGU], G.off[K_DN], &lo, &hi);
+      sm->xg_w0[u & 1] = (int)(lo % kConsumerWarps);
+      sm->xg_n[u & 1] = (int)(hi - lo);
+      local_range(G, u, G.off[K_DN], G.off[K_COUNT], &lo, &hi);
+      sm->xd_w0[u & 1] = (int)(lo % kConsumerWarps);
+      sm->xd_n[u & 1] = (int)(hi - lo);
     }
     __syncwarp();
     if (lane == 0) signal_ready(&sm->x_ready, &sm->x_bar, u);
-    // the eighths of the x transform that no consumer warp will do (warps without a gate/up
-    // chunk of this unit)
-    if (gu_on) {
-      unsigned lo, hi;
-      local_range(G, u, G.off[K_SGU], G.off[K_DN], &lo, &hi);
-      int done = 0;
-      for (int w = 0; w < kConsumerWarps; ++w)
-        if (!warp_in_range(lo, hi, w))
-          done += transform_share(XA, XG, G.H / 32, w, G.bits, [&](int) { return f; });
-      if (done && lane == 0) red_release_cta_smem(&sm->xg_done[u & 1], (unsigned)done);
-    }
     // ---- routing decision: needs every router chunk of unit u
     float sigma = 1.f;
     if (G.route_on) {
@@ -1017,15 +1016,6 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
         break;
       __syncwarp();
       if (lane == 0) signal_ready(&sm->xd_ready, &sm->xd_bar, u);
-      // the eighths of the down-input transform that no consumer warp will do
-      unsigned lo, hi;
-      local_range(G, u, G.off[K_DN], G.off[K_COUNT], &lo, &hi);
-      int done = 0;
-      for (int w = 0; w < kConsumerWarps; ++w)
-        if (!warp_in_range(lo, hi, w))
-          done += transform_share(XA, XA, G.nseg * (G.I / 32), w, G.bits,
-                                  [&](int t) { return xd_scale(G, sm, u, t); });
-      if (done && lane == 0) red_release_cta_smem(&sm->xd_done[u & 1], (unsigned)done);
     }
   }
 }
@@ -1355,7 +1345,9 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
       if (xd_mine != need) {
         xd_mine = need;
         share_wait = true;
-        const int d = transform_share(XA, XA, G.nseg * (G.I / 32), w, G.bits,
+        int n_sh;
+        const int rk = share_rank(sm->xd_w0[cv.u & 1], sm->xd_n[cv.u & 1], w, &n_sh);
+        const int d = transform_share(XA, XA, G.nseg * (G.I / 32), rk, n_sh, G.bits,
                                       [&](int t) { return xd_scale(G, sm, cv.u, t); });
         if (lane == 0 && d) red_release_cta_smem(&sm->xd_done[cv.u & 1], (unsigned)d);
       }
@@ -1368,7 +1360,9 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, i
         xg_mine = need;
         share_wait = true;
         const float f = sm->xf[cv.u & 1];
-        const int d = transform_share(XA, XG, G.H / 32, w, G.bits,
+        int n_sh;
+        const int rk = share_rank(sm->xg_w0[cv.u & 1], sm->xg_n[cv.u & 1], w, &n_sh);
+        const int d = transform_share(XA, XG, G.H / 32, rk, n_sh, G.bits,
                                       [&](int) { return f; });
         if (lane == 0 && d) red_release_cta_smem(&sm->xg_done[cv.u & 1], (unsigned)d);
       }

@@ -12,10 +12,11 @@
 // Completion is counted per class: CL_ROUTER (router chunks), CL_GU (shared and routed gate/
 // up chunks) and CL_DN. Chunk g of the launch (g = unit * chunks_per_unit + index) belongs to
 // CTA g mod gridDim; inside a CTA, local chunk i goes to consumer warp i mod kConsumerWarps and
-// ring stage i mod nstage. The transforms of a unit's x and down input are shared: each
-// consumer warp does one eighth at its first chunk that needs it, then waits for the other
-// eighths; those first chunks are at most kConsumerWarps - 1 local chunks apart, and the ring
-// holds at least kConsumerWarps stages, so they are all in flight together. Every other wait
+// ring stage i mod nstage. The transforms of a unit's x and down input are shared by the
+// consumer warps that hold the unit's gate/up (down) chunks, an equal part each, done at the
+// warp's first chunk that needs it, after which it waits for the other parts; those first
+// chunks are at most kConsumerWarps - 1 local chunks apart, and the ring holds at least
+// kConsumerWarps stages, so they are all in flight together. Every other wait
 // a chunk makes is on chunks with smaller g, so with all CTAs resident (one per SM) the
 // schedule cannot deadlock, and every wait is bounded in time.
 #pragma once
