@@ -14,7 +14,7 @@
 //   with the scale and bias factored out of the slice sum (same value in real arithmetic;
 //     "Qu'est-ce que Flash-MoE ?" (a2a-mcp.org, fr), §2 "Noyaux de Déquantification Optimisés
 //      pour FMA"); sum(q*x) is taken as integer dot products of the codes with three 8-bit
-//   digit planes of x (x ~ s_x (d0 + d1/128 + d2/16384), within 3.5e-7 of the slice's largest
+//   digit planes of x (x ~ s_x (d0 + d1/128 + d2/16384), within 1e-6 of the slice's largest
 //   |x|), so that one dp4a covers four weights.
 //
 // How: one CTA per SM, every CTA working through a static share of every unit's chunks.
@@ -856,17 +856,22 @@ __device__ __forceinline__ constexpr int digit_col(int n, int b) {
 }
 
 // The digit form of one 32-value slice v (already scaled): scale s = max|v| / 127 and the
-// digits of v/s, so that v ~ s * (d0 + d1/128 + d2/16384) to within 2.4e-7 * max|v|. Chunk
+// digits of v/s, so that v ~ s * (d0 + d1/128 + d2/16384) to within 1e-6 * max|v|. Chunk
 // i < 6 of the slice (at xpos(t, i)) holds digit plane i/2, words 4(i%2) .. 4(i%2)+3; chunk 6
 // holds {s, sum of v}.
 template <int BITS>
 __device__ __forceinline__ void store_digits(const float (&v)[32], float* xt, int t) {
-  float m = 0.f, sum = 0.f;
+  float mq[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains each
 #pragma unroll
-  for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
-#pragma unroll
-  for (int j = 0; j < 32; j += 4) sum += (v[j] + v[j + 1]) + (v[j + 2] + v[j + 3]);
-  const float k = m > 0.f ? 2080768.f / m : 0.f;  // 127 * 2^14 / max|v|
+  for (int j = 0; j < 32; ++j) {
+    mq[j & 3] = fmaxf(mq[j & 3], fabsf(v[j]));
+    sq[j & 3] += v[j];
+  }
+  const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+  const float sum = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+  // 127 * 2^14 / max|v|; a few ulp of error in k only shift |q| by a few units near its
+  // limit, which the digit ranges absorb, and the scale below is taken from m directly
+  const float k = m > 0.f ? __fdividef(2080768.f, m) : 0.f;
   uint32_t w[3][8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) {
