@@ -24,11 +24,12 @@
 //                   input), selects the top-K experts once the router is complete, and brings
 //                   in the down input [h_s | h_k] once every gate/up chunk is complete;
 //   consumer warps  each owns whole chunks (local chunk i -> warp i mod kConsumerWarps); each
-//                   puts one eighth of the unit's x and of its down input [sigma*h_s | w_k*h_k]
-//                   into digit form; cuts codes into bytes (nibbles or bit-planes) for dp4a
-//                   against the digit planes, reduces its row sums inside the warp and runs the
-//                   chunk's epilogue (logit store, SwiGLU, or residual + combine) itself -- no
-//                   block-wide barrier and no cross-warp reduction on the hot path.
+//                   puts its part of the unit's x and of its down input
+//                   [sigma*h_s | w_k*h_k] into digit form; cuts codes into bytes (nibbles or
+//                   bit-planes) for dp4a against the digit planes, reduces its row sums
+//                   inside the warp and runs the chunk's epilogue (logit store, SwiGLU, or
+//                   residual + combine) itself -- no block-wide barrier and no cross-warp
+//                   reduction on the hot path.
 // Completion is counted per run of same-class chunks of a CTA: the warp finishing a CTA's run
 // makes one gpu-scope release-acquire atomic on the class counter, and the stager warps poll
 // that counter (it is performed in L2, so no second hop is needed). Every spin-wait is
@@ -199,8 +200,8 @@ struct Smem {  // small shared state (in the misc area)
   uint64_t xd_bar;             // raw down input [h_s | h_k] of the unit in XA
   unsigned x_ready, rt_ready, xd_ready;
   // The transforms of x (into XG) and of the down input (in place in XA) are shared by the
-  // consumer warps: one eighth each (the stager does the eighths of warps that have no chunk
-  // needing them); per unit parity, the number of slices transformed so far.
+  // consumer warps holding the unit's chunks that need them; per unit parity, the number of
+  // slices transformed so far.
   unsigned xg_done[2], xd_done[2];
   // per unit parity: the warps holding the unit's gate/up (down) chunks share its x (down
   // input) transform; the first of them (local chunk index mod 8) and how many chunks there are
