@@ -89,7 +89,10 @@ def test_layer_tiny_without_shared_or_gate(fmoe, orc, shared, gate):
 
 
 @pytest.mark.parametrize("shape", [(192, 320, 7, 3, 4), (64, 64, 1, 1, 2), (128, 64, 40, 8, 4),
-                                   (1024, 576, 33, 5, 2)])
+                                   (1024, 576, 33, 5, 2),
+                                   # more than 512 experts: the top-K keeps 16 keys per lane
+                                   # across passes of 512 (a merge per pass)
+                                   (128, 64, 1100, 8, 4), (256, 128, 513, 2, 2)])
 def test_layer_odd_shapes(fmoe, orc, shape):
     H, I, E, K, bits = shape
     wl = wl_variant("tiny", H=H, I=I, E=E, K=K, bits=bits)
