@@ -176,12 +176,6 @@ __device__ __forceinline__ unsigned count_cong(unsigned long long lo, unsigned l
   return (unsigned)(b - a);
 }
 
-// chunks of class `cls` of unit u that belong to this CTA
-__device__ __forceinline__ unsigned run_len(const Geo& G, int u, int cls) {
-  const unsigned long long base = (unsigned long long)u * (unsigned)G.off[K_COUNT];
-  return count_cong(base + class_lo(G, cls), base + class_hi(G, cls), blockIdx.x, gridDim.x);
-}
-
 __device__ __forceinline__ unsigned local_chunks(const Prog& P, const Geo& G) {
   const unsigned long long total = (unsigned long long)P.n_units * (unsigned)G.off[K_COUNT];
   return count_cong(0ull, total, blockIdx.x, gridDim.x);
@@ -206,6 +200,7 @@ struct Smem {  // small shared state (in the misc area)
   // per unit parity: the warps holding the unit's gate/up (down) chunks share its x (down
   // input) transform; the first of them (local chunk index mod 8) and how many chunks there are
   int xg_w0[2], xg_n[2], xd_w0[2], xd_n[2];
+  unsigned run_n[2][CL_COUNT];  // per unit parity: this CTA's chunks of each class
   float xf[2];                 // RMSNorm factor of the unit's x (1 without a norm)
   float sigma[2];              // sigmoid(g . x) of the unit (1 without a shared gate)
   volatile int abort;
@@ -364,7 +359,7 @@ __device__ __forceinline__ void finish_run(const Prog& P, const Geo& G, Smem* sm
   __syncwarp();
   if ((threadIdx.x & 31) == 0) {
     const unsigned old = atom_add_acq_rel_cta_smem(&sm->run_cnt[cls], mine);
-    const unsigned nrun = run_len(G, u, cls);
+    const unsigned nrun = sm->run_n[u & 1][cls];  // recorded by the stager before x(u)
     if (old + mine == nrun) {
       atom_exch_cta_smem(&sm->run_cnt[cls], 0u);
       if (!(cls == CL_ROUTER && (P.debug & 1)))
@@ -982,9 +977,13 @@ __device__ void stager(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
       local_range(G, u, G.off[K_SGU], G.off[K_DN], &lo, &hi);
       sm->xg_w0[u & 1] = (int)(lo % kConsumerWarps);
       sm->xg_n[u & 1] = (int)(hi - lo);
+      sm->run_n[u & 1][CL_GU] = hi - lo;
       local_range(G, u, G.off[K_DN], G.off[K_COUNT], &lo, &hi);
       sm->xd_w0[u & 1] = (int)(lo % kConsumerWarps);
       sm->xd_n[u & 1] = (int)(hi - lo);
+      sm->run_n[u & 1][CL_DN] = hi - lo;
+      local_range(G, u, G.off[K_ROUTER], G.off[K_SGU], &lo, &hi);
+      sm->run_n[u & 1][CL_ROUTER] = hi - lo;
     }
     __syncwarp();
     if (lane == 0) signal_ready(&sm->x_ready, &sm->x_bar, u);
