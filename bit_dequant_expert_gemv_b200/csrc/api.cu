@@ -364,22 +364,28 @@ int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int 
 }
 
 int fmoe_sync_status(void* stream) {
-  DevState* d;
-  int rc = dev_state(&d);
-  if (rc) return rc;
-  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-  int v = 0;
-  CK(cudaMemcpy(&v, d->err, sizeof v, cudaMemcpyDeviceToHost));
-  if (v != 0) CK(cudaMemset(d->err, 0, sizeof(int)));
+  // Reads the error words of whatever this library has set up on the current device and
+  // creates nothing: a caller that only uses fmoe_moe_layer_noalloc must not see the pooled
+  // path's error word or memory pool allocated here.
   int dev = 0;
   CK(cudaGetDevice(&dev));
-  if (g_na[dev].init) {  // the fixed-scratch entry point keeps its own error word
-    int* na_err = reinterpret_cast<int*>(g_na[dev].base + kNoAllocErrOff);
-    int w = 0;
-    CK(cudaMemcpy(&w, na_err, sizeof w, cudaMemcpyDeviceToHost));
-    if (w != 0) {
-      CK(cudaMemset(na_err, 0, sizeof(int)));
-      if (v == 0) v = w;
+  if (dev < 0 || dev >= 64) return fail(FMOE_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  int* pooled_err = nullptr;
+  int* na_err = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev[dev].init) pooled_err = g_dev[dev].err;
+    if (g_na[dev].init) na_err = reinterpret_cast<int*>(g_na[dev].base + kNoAllocErrOff);
+  }
+  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  for (int* w : {pooled_err, na_err}) {
+    if (!w) continue;
+    int x = 0;
+    CK(cudaMemcpy(&x, w, sizeof x, cudaMemcpyDeviceToHost));
+    if (x != 0) {
+      CK(cudaMemset(w, 0, sizeof(int)));
+      if (v == 0) v = x;
     }
   }
   if (v == 0) return FMOE_OK;

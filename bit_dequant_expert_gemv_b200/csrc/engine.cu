@@ -633,17 +633,13 @@ __device__ __forceinline__ double unit_logit(const Geo& G, const double* lg, int
   return a;
 }
 
-// Order-preserving 32-bit key of a binary32 value (larger value <=> larger signed key).
-__device__ __forceinline__ int fkey(float f) {
-  const int b = __float_as_int(f);
-  return b >= 0 ? b : b ^ 0x7FFFFFFF;
-}
-
 // Top-K over at most 512 experts by one warp (lane l holds experts l + 32 i). K rounds: the
-// warp maximum of the lanes' best 32-bit keys (the logit rounded to binary32), then the lowest
-// expert index holding it, so that ties go to the lower index; logits that differ by less than
-// binary32 resolution (~6e-8 relative, far inside the tie band of the routing decision) count
-// as tied. The winners' binary64 logits are carried along for the weights
+// warp maximum of the lanes' best packed keys (pkey: the binary64 logit's order-preserving key
+// with its 13 lowest bits replaced by 8191 - e, so that one unsigned compare orders by logit and
+// breaks ties toward the lower index; logits within ~2^-39 relative of each other count as
+// tied, far inside the 1e-6 band where either order is correct, at any logit magnitude), taken
+// as two 32-bit warp reductions (high word, then low word among the lanes holding that high
+// word). The winners' binary64 logits are carried along for the weights
 // w_k = exp(l_k - l_max) / sum_sel exp(l_j - l_max): the softmax over all experts followed by
 // renormalisation over the selected ones, where the full softmax denominator cancels.
 __device__ void topk_warp_512(const Geo& G, const double* lg, const float* bias, int* rt_e,
@@ -664,37 +660,40 @@ __device__ void topk_warp_512(const Geo& G, const double* lg, const float* bias,
   for (int sg = 2; sg < G.rseg; ++sg) {
     double part[kPer];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      part[i] = __ldcg(lg + (size_t)sg * G.nr + min(lane + 32 * i, G.E - 1));
+    for (int i = 0; i < kPer; ++i) part[i] = __ldcg(lg + (size_t)sg * G.nr + min(lane + 32 * i, G.E - 1));
 #pragma unroll
     for (int i = 0; i < kPer; ++i) lv[i] += part[i];
   }
-  int key[kPer];
+  unsigned long long key[kPer];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) key[i] = lane + 32 * i < G.E ? fkey((float)lv[i]) : INT_MIN;
-  // the lane's best: largest key, lowest index on ties
-  auto lane_best = [&](int& bk, int& bi) {
+  for (int i = 0; i < kPer; ++i) key[i] = lane + 32 * i < G.E ? pkey(lv[i], lane + 32 * i) : 0ull;
+  // the lane's best: largest key (the lowest index among equal logits by construction)
+  auto lane_best = [&](unsigned long long& bk, int& bi) {
     bk = key[0];
     bi = 0;
 #pragma unroll
     for (int i = 1; i < kPer; ++i)
       if (key[i] > bk) bk = key[i], bi = i;
   };
-  int bk, bi;
+  unsigned long long bk;
+  int bi;
   lane_best(bk, bi);
   int sel_e = 0;
   double sel_l = 0.0;
   for (int k = 0; k < G.K; ++k) {
-    const int mk = __reduce_max_sync(0xffffffffu, bk);
-    const int we = (int)__reduce_min_sync(0xffffffffu, bk == mk ? (unsigned)(lane + 32 * bi) : 0xFFFFFFFFu);
-    const bool win = lane == (we & 31);
+    const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(bk >> 32));
+    const unsigned lo =
+        __reduce_max_sync(0xffffffffu, (unsigned)(bk >> 32) == hi ? (unsigned)bk : 0u);
+    const unsigned long long win = ((unsigned long long)hi << 32) | lo;
+    const int we = 0x1FFF - (int)(win & 0x1FFFull);  // winning expert
+    const bool mine_w = bk == win && win != 0ull;     // exactly one lane holds it
     double wl = 0.0;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) wl = (win && i == bi) ? lv[i] : wl;
+    for (int i = 0; i < kPer; ++i) wl = (mine_w && i == bi) ? lv[i] : wl;
     wl = __shfl_sync(0xffffffffu, wl, we & 31);
-    if (win) {
+    if (mine_w) {
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) key[i] = i == bi ? INT_MIN : key[i];
+      for (int i = 0; i < kPer; ++i) key[i] = i == bi ? 0ull : key[i];
       lane_best(bk, bi);
     }
     if (lane == k) {
@@ -1443,8 +1442,26 @@ extern "C" cudaError_t fmoe_engine_configure(int max_smem) {
                               max_smem);
 }
 
+// The CTAs of one launch wait on each other's progress, so they must all be resident at
+// once: the launch is cooperative, which makes a grid that cannot be co-resident a launch
+// error instead of a wait that runs out of budget.
 extern "C" cudaError_t fmoe_engine_launch(const fmoe::Prog* P, const fmoe::Geo* G, int grid,
                                           cudaStream_t stream) {
-  fmoe::engine_kernel<<<grid, fmoe::kThreads, G->smem_bytes, stream>>>(*P, *G);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)fmoe::kThreads);
+  cfg.dynamicSmemBytes = G->smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fmoe::engine_kernel, *P, *G);
+}
+
+// CTAs of the engine kernel that fit on one SM with `smem` bytes of dynamic shared memory.
+extern "C" cudaError_t fmoe_engine_occupancy(int smem, int* ctas_per_sm) {
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, fmoe::engine_kernel,
+                                                       fmoe::kThreads, (size_t)smem);
 }

@@ -30,22 +30,37 @@ def _layer_inputs(fmoe, name, t):
 
 
 @pytest.mark.parametrize("name", ["tiny", "full_q4_natural", "full_q2"])
-def test_noalloc_matches_layer(fmoe, name):
+def test_noalloc_matches_layer(fmoe, orc, name):
+    from oracle.workload import HostLayer
+    from gpu_helpers import check_routing
     wl, dl, x, res = _layer_inputs(fmoe, name, 3)
     K = wl.K
     idx_ref = torch.empty(K, dtype=torch.int32, device="cuda")
     w_ref = torch.empty(K, dtype=torch.float32, device="cuda")
     ref = fmoe.moe_layer(dl.desc, x, res, None, idx=idx_ref, weight=w_ref)
     assert fmoe.sync_status() == 0
-    for call in range(2):  # two calls in a row reuse the same fixed scratch
-        out = torch.full_like(x, float("nan"))
-        idx = torch.full((K,), -1, dtype=torch.int32, device="cuda")
-        w = torch.full((K,), float("nan"), dtype=torch.float32, device="cuda")
-        fmoe.moe_layer_noalloc(dl.desc, x, res, None, out=out, idx=idx, weight=w)
+    outs = [torch.full_like(x, float("nan")) for _ in range(3)]
+    idxs = [torch.full((K,), -1, dtype=torch.int32, device="cuda") for _ in range(3)]
+    ws = [torch.full((K,), float("nan"), dtype=torch.float32, device="cuda") for _ in range(3)]
+    free_before = None
+    for call in range(3):  # calls in a row reuse the same fixed scratch
+        fmoe.moe_layer_noalloc(dl.desc, x, res, None, out=outs[call], idx=idxs[call],
+                               weight=ws[call])
         assert fmoe.sync_status() == 0, fmoe.last_error()
-        check_out(out.cpu().numpy(), ref.cpu().numpy(), f"{name} call {call}")
-        assert idx.cpu().tolist() == idx_ref.cpu().tolist()
-        assert np.abs(w.cpu().numpy() - w_ref.cpu().numpy()).max() <= W_TOL
+        if call == 0:  # the first call on the device did the set-up; later calls allocate nothing
+            free_before = torch.cuda.mem_get_info()[0]
+    assert torch.cuda.mem_get_info()[0] == free_before
+    # the oracle, for the same token
+    hl = HostLayer(orc, wl, 0)
+    xh, rh = x.cpu().numpy(), res.cpu().numpy()
+    want, oi, ow, logits = hl.forward(xh, rh)
+    for call in range(3):
+        out, idx, w = outs[call].cpu().numpy(), idxs[call].cpu().numpy(), ws[call].cpu().numpy()
+        check_out(out, ref.cpu().numpy(), f"{name} call {call} vs fmoe_moe_layer")
+        assert idx.tolist() == idx_ref.cpu().tolist()
+        assert np.abs(w - w_ref.cpu().numpy()).max() <= W_TOL
+        assert check_routing(idx, w, logits, K)
+        check_out(out, want, f"{name} call {call} vs oracle")
 
 
 def test_noalloc_rejects_oversized_scratch(fmoe):
