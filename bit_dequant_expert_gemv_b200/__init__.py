@@ -51,7 +51,8 @@ _SIGS = {
                                           C.c_void_p]),
     "fmoe_stack_graph_launch": (C.c_int, [C.c_void_p, C.c_void_p]),
     "fmoe_stack_graph_destroy": (C.c_int, [C.c_void_p]),
-    "fmoe_describe_geometry": (C.c_int, [C.c_int] * 7 + [C.c_void_p, C.c_int]),
+    "fmoe_describe_geometry": (C.c_int, [C.c_int] * 8 + [C.c_void_p, C.c_int]),
+    "fmoe_set_dot_form": (C.c_int, [C.c_int]),
     "fmoe_launch_count": (C.c_uint64, []),
 }
 _lib = None
@@ -128,16 +129,24 @@ def expert_bytes(hidden: int, inter: int, bits: int) -> int:
     return int(lib().fmoe_expert_bytes(hidden, inter, bits))
 
 
-def describe_geometry(H, I, E, K, bits, flags=15, max_smem=232448) -> dict:
-    names = ("H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr rseg "
-             "rcols rrows nrb R nb nseg Rd n0 n1 n2 n3 off0 off1 off2 off3 off4 ncl0 ncl1 ncl2 "
-             "gu_nsl gu_S gu_P gu_nrl dn_nsl dn_S dn_P dn_nrl stage_bytes nstage o_ring o_full "
-             "o_empty o_xa o_xg o_red o_misc smem_bytes").split()
-    buf = (C.c_int64 * len(names))()
-    n = lib().fmoe_describe_geometry(H, I, E, K, bits, flags, max_smem, buf, len(names))
+GEOMETRY_FIELDS = ("H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr "
+                   "rseg rcols rrows au hr ad dr nseg sh wh gh si wi pi ji stage_bytes nA nB "
+                   "o_ringA o_ringB o_x o_h o_red o_oacc o_misc o_bar oacc_n smem_bytes "
+                   "consumer_warps max_rows_thread max_rows_warp red_slot").split()
+
+
+def describe_geometry(H, I, E, K, bits, flags=15, max_smem=232448, sms=148) -> dict:
+    buf = (C.c_int64 * len(GEOMETRY_FIELDS))()
+    n = lib().fmoe_describe_geometry(H, I, E, K, bits, flags, max_smem, sms, buf,
+                                     len(GEOMETRY_FIELDS))
     if n < 0:
         raise FmoeError("fmoe_describe_geometry", n, last_error())
-    return {k: int(buf[i]) for i, k in enumerate(names[:n])}
+    return {k: int(buf[i]) for i, k in enumerate(GEOMETRY_FIELDS[:n])}
+
+
+def set_dot_form(form: int):
+    """0: digit planes + dp4a (default), 1: literal fma(q, s*x, z*x), 2: naive (q*s + z)*x."""
+    _ck("fmoe_set_dot_form", lib().fmoe_set_dot_form(int(form)))
 
 
 def launch_count() -> int:

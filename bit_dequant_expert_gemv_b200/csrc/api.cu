@@ -17,6 +17,7 @@
 extern "C" cudaError_t fmoe_engine_launch(const fmoe::Prog* P, const fmoe::Geo* G, int grid,
                                           cudaStream_t stream);
 extern "C" cudaError_t fmoe_engine_configure(int max_smem);
+extern "C" cudaError_t fmoe_engine_occupancy(int smem, int* ctas_per_sm);
 extern "C" cudaError_t fmoe_pack_launch(const float* w, int rows, int cols, int bits, void* dst,
                                         int sms, cudaStream_t stream);
 
@@ -28,6 +29,8 @@ thread_local std::string g_err;
 thread_local uint64_t g_launches = 0;
 thread_local uint64_t g_wait_ns = 1000000000ull;
 thread_local int g_debug = 0;
+thread_local int g_form = FORM_DIGITS;
+constexpr int kMaxUnits = 1 << 24;  // units per launch (chunk and signal counters stay in range)
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -93,6 +96,10 @@ int dev_state(DevState** out) {
     uint64_t keep = 64ull << 20;  // keep up to 64 MiB of scratch cached between calls
     CK(cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep));
     CK(fmoe_engine_configure(d.max_smem));
+    int per_sm = 0;
+    CK(fmoe_engine_occupancy(d.max_smem, &per_sm));
+    if (per_sm < 1)
+      return fail(FMOE_ERR_UNSUPPORTED, "the engine kernel does not fit one SM (%d CTAs)", per_sm);
     d.init = true;
   }
   *out = &d;
@@ -108,18 +115,10 @@ int rows_for_16(unsigned row_bytes) {
   return r;
 }
 
-// Lane layout of a chunk whose (virtual) rows have nsl 32-column slices and nrows rows.
-LaneMap lane_map(int nsl, int nrows) {
-  LaneMap m;
-  m.nsl = nsl;
-  m.S = 32;
-  if (nsl < 32) {
-    m.S = 1;
-    while (m.S < nsl) m.S <<= 1;
-  }
-  m.P = 32 / m.S;
-  m.nrl = (nrows + m.P - 1) / m.P;
-  return m;
+int pow2ceil(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
 }
 
 // ---------------------------------------------------------------- validation and geometry
@@ -135,11 +134,10 @@ int check_shape(int H, int I, int E, int K, int bits) {
   return FMOE_OK;
 }
 
-// Chunk sizes, lane layouts and the shared-memory carve-up of one launch. Each chunk kind
-// takes as many rows as fit kStageTarget bytes (at least one aligned group of rows), within
-// what one warp's lanes accumulate (kRowsPerLane rows per lane).
+// Chunk sizes, consumer thread layouts and the shared-memory carve-up of one launch on a GPU
+// with `sms` SMs (one CTA each) and `max_smem` bytes of shared memory per CTA.
 int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on, bool routed_on,
-             bool gate_on, int max_smem, Geo* G) {
+             bool gate_on, int max_smem, int sms, Geo* G) {
   memset(G, 0, sizeof *G);
   G->H = H; G->I = I; G->E = E; G->K = K; G->bits = bits;
   G->route_on = route_on; G->shared_on = shared_on; G->routed_on = routed_on;
@@ -147,91 +145,106 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   G->rc_h = (unsigned)H * bits / 8; G->rs_h = (unsigned)H / 16;
   G->rc_i = (unsigned)I * bits / 8; G->rs_i = (unsigned)I / 16;
   G->q_gu = (unsigned long long)I * (G->rc_h + G->rs_h);
-  const unsigned cap = (unsigned)kStageTarget;
-  // router: whole rows when a row fits, else column segments of one row
+  if (sms < 1) return fail(FMOE_ERR_INVALID, "SM count %d", sms);
+  const bool gu_on = shared_on || routed_on;
+  G->nseg = (shared_on ? 1 : 0) + (routed_on ? K : 0);
+  G->au = rows_for_16(G->rs_h);
+  G->ad = rows_for_16(G->rs_i);
+  // a stage holds at least one aligned group of gate + up rows and of down rows
+  const unsigned stage = align_up(
+      std::max({kStage, gu_on ? 2u * (unsigned)G->au * (G->rc_h + G->rs_h) : 0u,
+                G->nseg > 0 ? (unsigned)G->ad * (G->rc_i + G->rs_i) : 0u}),
+      128);
+  G->stage_bytes = stage;
+  // router: whole rows when a row fits kStage bytes, else column segments of one row
   G->nr = route_on ? E + (G->gate_on ? 1 : 0) : 0;
-  if (4u * H <= cap) {
+  if (4u * H <= kStage) {
     G->rseg = 1;
     G->rcols = H;
-    G->rrows = std::max(1, std::min(64, (int)(cap / (4u * H))));
+    G->rrows = std::max(1, std::min(32, (int)(kStage / (4u * H))));
   } else {
-    int d = (int)((4u * H + cap - 1) / cap);
+    int d = (int)((4u * H + kStage - 1) / kStage);
     while (H % d || (H / d) % 4) ++d;
     G->rseg = d;
     G->rcols = H / d;
     G->rrows = 1;
   }
-  G->nrb = G->nr ? (G->nr + G->rrows - 1) / G->rrows : 0;
-  // gate/up: R rows of gate and R of up per chunk
+  // gate/up: thread layout, then hr h-rows (gate + up) per chunk
+  G->sh = H / 32;
+  G->wh = G->sh <= 32 ? pow2ceil(G->sh) : 32 * ((G->sh + 31) / 32);
+  G->gh = kConsumers / G->wh;
   {
-    const int al = std::max(rows_for_16(G->rc_h), rows_for_16(G->rs_h));
-    const LaneMap m1 = lane_map(H / 32, 1);
-    int r = (int)(cap / (2u * (G->rc_h + G->rs_h)));
-    r = std::min(r, kRowsPerLane * m1.P / 2);
-    r = std::min(r, I);
-    r = std::max(al, r / al * al);
-    G->R = r;
-    G->nb = (I + r - 1) / r;
-    G->gu = lane_map(H / 32, 2 * r);
+    int hr = (int)(stage / (2u * (G->rc_h + G->rs_h)));
+    hr = std::min(hr, kMaxHr);
+    hr = std::min(hr, I);
+    hr = std::min(hr, kMaxRowsThread * G->gh / 2);
+    hr = hr / G->au * G->au;
+    if (!gu_on) hr = G->au;  // no gate/up rows in this launch
+    if (hr < G->au) return fail(FMOE_ERR_UNSUPPORTED, "gate/up rows do not fit a stage (H=%d)", H);
+    G->hr = hr;
   }
-  // down: Rd virtual rows of nseg segments per chunk
-  G->nseg = (shared_on ? 1 : 0) + (routed_on ? K : 0);
-  if (G->nseg > 0) {
-    const int al = std::max(rows_for_16(G->rc_i), rows_for_16(G->rs_i));
-    const LaneMap m1 = lane_map(G->nseg * I / 32, 1);
-    int r = (int)(cap / ((unsigned)G->nseg * (G->rc_i + G->rs_i)));
-    r = std::min(r, kRowsPerLane * m1.P);
-    r = std::min(r, H);
-    r = std::max(al, r / al * al);
-    G->Rd = r;
-    G->dn = lane_map(G->nseg * I / 32, r);
+  // down: lane layout, then dr output rows per chunk
+  G->si = I / 32;
+  if (G->si <= 32) {
+    G->wi = pow2ceil(G->si);
+    G->pi = 32 / G->wi;
+    G->ji = 1;
+  } else {
+    G->wi = 32;
+    G->pi = 1;
+    G->ji = (G->si + 31) / 32;
   }
-  if (G->gu.nrl > kRowsPerLane || G->dn.nrl > kRowsPerLane)
-    return fail(FMOE_ERR_UNSUPPORTED, "row layout too wide (H=%d I=%d K=%d)", H, I, K);
-  G->n[K_ROUTER] = route_on ? G->nrb * G->rseg : 0;
-  G->n[K_SGU] = shared_on ? G->nb : 0;
-  G->n[K_RGU] = routed_on ? K * G->nb : 0;
-  G->n[K_DN] = G->nseg > 0 ? (H + G->Rd - 1) / G->Rd : 0;
-  G->off[0] = 0;
-  for (int k = 0; k < K_COUNT; ++k) G->off[k + 1] = G->off[k] + G->n[k];
-  if (G->off[K_COUNT] == 0) return fail(FMOE_ERR_INVALID, "nothing to compute");
-  G->ncl[CL_ROUTER] = G->n[K_ROUTER];
-  G->ncl[CL_GU] = G->n[K_SGU] + G->n[K_RGU];
-  G->ncl[CL_DN] = G->n[K_DN];
-  unsigned stage = 0;
-  if (route_on) stage = std::max(stage, (unsigned)G->rrows * 4u * G->rcols);
-  if (shared_on || routed_on) stage = std::max(stage, 2u * G->R * (G->rc_h + G->rs_h));
-  if (G->nseg > 0) stage = std::max(stage, (unsigned)G->Rd * G->nseg * (G->rc_i + G->rs_i));
-  G->stage_bytes = align_up(stage, 128);
-  // fixed areas after the ring
+  {
+    int dr = (int)(stage / (G->rc_i + G->rs_i));
+    dr = std::min(dr, kMaxRowsWarp * kConsumerWarps * G->pi);
+    dr = std::min(dr, H);
+    dr = dr / G->ad * G->ad;
+    if (G->nseg == 0) dr = G->ad;  // no down rows in this launch
+    if (dr < G->ad) return fail(FMOE_ERR_UNSUPPORTED, "down rows do not fit a stage (I=%d)", I);
+    G->dr = dr;
+  }
+  {
+    const int nu = H / G->ad;
+    G->oacc_n = G->nseg > 0 ? ((nu + sms - 1) / sms) * G->ad : 0;
+  }
+  // shared memory: ring A | ring B | x | h | reductions | output accumulators | misc | barriers
   unsigned o = 0;
   auto take = [&](unsigned bytes) {
     unsigned at = o;
     o = align_up(o + bytes, 128);
     return at;
   };
-  // x (raw) / down input (digit form); x in digit form: 128 bytes per 32-column slice either way
-  G->o_xa = take(4u * (unsigned)std::max(H, G->nseg * I));
-  G->o_xg = take(4u * H);
-  G->o_red = take(4u * kConsumerWarps * 16 * kRowsPerLane);   // per-warp row sums
-  G->o_misc = take(512);
-  const unsigned fixed = o;
-  const unsigned avail = (unsigned)max_smem;
-  // at least one stage per consumer warp: the first chunks of a unit that need a shared
-  // transform (one per warp) must all fit in the ring at once
-  if (fixed + kConsumerWarps * (G->stage_bytes + 16) > avail)
-    return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for %d stages", kConsumerWarps);
-  int ns = (int)((avail - fixed) / (G->stage_bytes + 16));
-  ns = std::min(ns, kMaxStages);
-  G->nstage = ns;
-  // final layout: ring | fixed areas | barriers
-  const unsigned ring = (unsigned)ns * G->stage_bytes;
-  G->o_ring = 0;
-  G->o_xa += ring; G->o_xg += ring; G->o_red += ring;
-  G->o_misc += ring;
-  G->o_full = ring + fixed;
-  G->o_empty = G->o_full + 8u * ns;
-  G->smem_bytes = G->o_empty + 8u * ns;
+  const unsigned x_b = 4u * (unsigned)H;
+  const unsigned h_b = 4u * (unsigned)(G->nseg * I);
+  const unsigned wn = G->wh > 32 ? (unsigned)G->wh / 32 : 1u;
+  const unsigned red_slot = std::max(8u * (unsigned)G->rrows * kConsumerWarps,
+                                     4u * 2u * (unsigned)G->hr * wn);
+  const unsigned oacc_b = 4u * (unsigned)std::max(G->oacc_n, 1);
+  const unsigned misc_b = 512;
+  const unsigned fixed = align_up(x_b, 128) + align_up(std::max(h_b, 128u), 128) +
+                         align_up(oacc_b, 128) + misc_b;
+  const unsigned per_stage = stage + red_slot + 16;
+  if ((unsigned)max_smem < fixed + 4 * per_stage + 256)
+    return fail(FMOE_ERR_UNSUPPORTED, "shared memory too small for 4 stages");
+  int ns = (int)(((unsigned)max_smem - fixed - 256) / per_stage);
+  const bool a_used = route_on || shared_on, b_used = routed_on;
+  int nb = b_used ? std::min(kMaxStages, a_used ? ns / 2 : ns - 1) : 1;
+  int na = std::min(kMaxStages, ns - nb);
+  if (na < 1 || (a_used && na < 2) || (b_used && nb < 2))
+    return fail(FMOE_ERR_UNSUPPORTED, "not enough stages (%d)", ns);
+  G->nA = na;
+  G->nB = nb;
+  G->o_ringA = take((unsigned)na * stage);
+  G->o_ringB = take((unsigned)nb * stage);
+  G->o_x = take(x_b);
+  G->o_h = take(std::max(h_b, 128u));
+  G->red_slot = red_slot;
+  G->o_red = take(red_slot * (unsigned)(na + nb));
+  G->o_oacc = take(oacc_b);
+  G->o_misc = take(misc_b);
+  G->o_bar = o;
+  o += 16u * (unsigned)(na + nb);
+  G->smem_bytes = o;
   if (G->smem_bytes > (unsigned)max_smem)
     return fail(FMOE_ERR_UNSUPPORTED, "shared memory layout too large (%u)", G->smem_bytes);
   return FMOE_OK;
@@ -264,7 +277,7 @@ size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 ScratchPlan plan_scratch(const Geo& G, int n_units) {
   ScratchPlan s;
   size_t o = 0;
-  s.off_ctrl = o; o = up256(o + 4 * C_WORDS);
+  s.off_ctrl = o; o = up256(o + 4 * (size_t)kCtrlWords);
   s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
   s.zero_bytes = o;
   s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.rseg, 1) * std::max(G.nr, 1));
@@ -299,9 +312,7 @@ void fill_layers(Prog* P, const fmoe_layer_desc* layers, int n) {
 int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, int sms,
                    cudaStream_t st) {
   CK(cudaMemsetAsync(base, 0, sp.zero_bytes, st));
-  const long long total = (long long)P->n_units * G.off[K_COUNT];
-  const int grid = (int)std::min<long long>(sms, std::max<long long>(1, total));
-  cudaError_t e = fmoe_engine_launch(P, &G, grid, st);
+  cudaError_t e = fmoe_engine_launch(P, &G, sms, st);
   if (e != cudaSuccess) return cuda_fail(e, "engine launch");
   ++g_launches;
   return FMOE_OK;
@@ -326,6 +337,7 @@ void base_prog(Prog* P, int mode) {
   P->mode = mode;
   P->wait_ns = g_wait_ns;
   P->debug = g_debug;
+  P->form = g_form;
 }
 
 }  // namespace
@@ -341,23 +353,28 @@ void fmoe_set_wait_budget_ns(uint64_t ns) { g_wait_ns = ns < 1000 ? 1000 : ns; }
 
 void fmoe_set_fault_injection(int flags) { g_debug = flags; }
 
+int fmoe_set_dot_form(int form) {
+  if (form < 0 || form >= FORM_COUNT) return fail(FMOE_ERR_INVALID, "dot form %d", form);
+  g_form = form;
+  return FMOE_OK;
+}
+
 uint64_t fmoe_launch_count(void) { return g_launches; }
 
 int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int bits, int flags,
-                           int max_smem, int64_t* out, int n_out) {
+                           int max_smem, int sms, int64_t* out, int n_out) {
   int rc = check_shape(hidden, inter, n_experts, top_k, bits);
   if (rc) return rc;
   Geo G;
   if ((rc = make_geo(hidden, inter, n_experts, top_k, bits, flags & 1, flags & 2, flags & 4,
-                     flags & 8, max_smem, &G)))
+                     flags & 8, max_smem, sms, &G)))
     return rc;
   const int64_t v[] = {G.H, G.I, G.E, G.K, G.bits, G.route_on, G.shared_on, G.routed_on,
                        G.gate_on, G.rc_h, G.rs_h, G.rc_i, G.rs_i, (int64_t)G.q_gu, G.nr, G.rseg,
-                       G.rcols, G.rrows, G.nrb, G.R, G.nb, G.nseg, G.Rd, G.n[0], G.n[1], G.n[2],
-                       G.n[3], G.off[0], G.off[1], G.off[2], G.off[3], G.off[4], G.ncl[0],
-                       G.ncl[1], G.ncl[2], G.gu.nsl, G.gu.S, G.gu.P, G.gu.nrl, G.dn.nsl, G.dn.S,
-                       G.dn.P, G.dn.nrl, G.stage_bytes, G.nstage, G.o_ring, G.o_full, G.o_empty,
-                       G.o_xa, G.o_xg, G.o_red, G.o_misc, G.smem_bytes};
+                       G.rcols, G.rrows, G.au, G.hr, G.ad, G.dr, G.nseg, G.sh, G.wh, G.gh, G.si,
+                       G.wi, G.pi, G.ji, G.stage_bytes, G.nA, G.nB, G.o_ringA, G.o_ringB, G.o_x,
+                       G.o_h, G.o_red, G.o_oacc, G.o_misc, G.o_bar, G.oacc_n, G.smem_bytes,
+                       kConsumerWarps, kMaxRowsThread, kMaxRowsWarp, G.red_slot};
   const int n = (int)(sizeof v / sizeof v[0]);
   for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
   return n < n_out ? n : n_out;
@@ -445,7 +462,8 @@ int fmoe_route(const float* x, const float* router, const float* logit_bias, int
   DevState* d;
   if ((rc = dev_state(&d))) return rc;
   Geo G;
-  if ((rc = make_geo(hidden, 64, n_experts, top_k, 4, true, false, false, false, d->max_smem, &G)))
+  if ((rc = make_geo(hidden, 64, n_experts, top_k, 4, true, false, false, false, d->max_smem,
+                     d->sms, &G)))
     return rc;
   Prog P;
   base_prog(&P, MODE_SEQ);
@@ -467,7 +485,8 @@ int fmoe_expert_gemv(const void* expert, int hidden, int inter, int bits, const 
   DevState* d;
   if ((rc = dev_state(&d))) return rc;
   Geo G;
-  if ((rc = make_geo(hidden, inter, 1, 1, bits, false, true, false, false, d->max_smem, &G)))
+  if ((rc = make_geo(hidden, inter, 1, 1, bits, false, true, false, false, d->max_smem, d->sms,
+                     &G)))
     return rc;
   Prog P;
   base_prog(&P, MODE_SEQ);
@@ -489,7 +508,7 @@ static int prep_layers(const fmoe_layer_desc* layers, int n_layers, DevState* d,
       return fail(FMOE_ERR_INVALID, "all layers must agree on having a shared expert / gate");
   const fmoe_layer_desc& L = layers[0];
   return make_geo(L.hidden, L.inter, L.n_experts, L.top_k, L.bits, true, shared, true,
-                  gate && shared, d->max_smem, G);
+                  gate && shared, d->max_smem, d->sms, G);
 }
 
 int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float* x,
@@ -501,7 +520,7 @@ int fmoe_moe_layer_seq(const fmoe_layer_desc* layers, int n_layers, const float*
   Geo G;
   if ((rc = prep_layers(layers, n_layers, d, &G))) return rc;
   if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
-  if ((long long)n_tokens * G.off[K_COUNT] > 0x7ffffff0ll) return fail(FMOE_ERR_UNSUPPORTED, "too many tokens");
+  if (n_tokens > kMaxUnits) return fail(FMOE_ERR_UNSUPPORTED, "more than %d tokens", kMaxUnits);
   if (!x || !out) return fail(FMOE_ERR_INVALID, "x and out are required");
   if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
     return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
@@ -629,8 +648,8 @@ static int stack_prog(const fmoe_layer_desc* layers, int n_layers, const float* 
   int rc = prep_layers(layers, n_layers, d, G);
   if (rc) return rc;
   if (n_tokens < 1) return fail(FMOE_ERR_INVALID, "n_tokens must be >= 1");
-  if ((long long)n_tokens * n_layers * G->off[K_COUNT] > 0x7ffffff0ll)
-    return fail(FMOE_ERR_UNSUPPORTED, "too many tokens x layers for one launch");
+  if ((long long)n_tokens * n_layers > kMaxUnits)
+    return fail(FMOE_ERR_UNSUPPORTED, "more than %d tokens x layers in one launch", kMaxUnits);
   if (!h_in || !h_out) return fail(FMOE_ERR_INVALID, "h_in and h_out are required");
   if (!aligned16(h_in) || !aligned16(h_out) || !aligned16(h_trace))
     return fail(FMOE_ERR_ALIGN, "h_in, h_out, h_trace must be 16-byte aligned");

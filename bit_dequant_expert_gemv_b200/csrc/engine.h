@@ -1,24 +1,25 @@
 // engine.h — host/device description of one launch of the MoE engine kernel.
 //
-// A launch runs a sequence of "units"; a unit is one MoE layer applied to one token. The work
-// of a unit is cut into chunks of one shared-memory stage each, listed in dependency order:
-//   K_ROUTER  a column segment of one or more router rows (fp32 weights, binary64 sums); the
-//             shared-gate vector is router row E
-//   K_SGU     R rows of the shared expert's gate matrix and the same R rows of its up matrix
-//   K_RGU     the same for routed expert k (needs the routing decision)
-//   K_DN      Rd output rows of the fused down projection: output row j is the dot product of
-//             the concatenated rows j of every active down matrix (shared expert first, then
-//             routed k = 0..K-1) with the concatenated inputs [sigma*h_s | w_0*h_0 | ...]
-// Completion is counted per class: CL_ROUTER (router chunks), CL_GU (shared and routed gate/
-// up chunks) and CL_DN. Chunk g of the launch (g = unit * chunks_per_unit + index) belongs to
-// CTA g mod gridDim; inside a CTA, local chunk i goes to consumer warp i mod kConsumerWarps and
-// ring stage i mod nstage. The transforms of a unit's x and down input are shared by the
-// consumer warps that hold the unit's gate/up (down) chunks, an equal part each, done at the
-// warp's first chunk that needs it, after which it waits for the other parts; those first
-// chunks are at most kConsumerWarps - 1 local chunks apart, and the ring holds at least
-// kConsumerWarps stages, so they are all in flight together. Every other wait
-// a chunk makes is on chunks with smaller g, so with all CTAs resident (one per SM) the
-// schedule cannot deadlock, and every wait is bounded in time.
+// A launch runs a sequence of "units"; a unit is one MoE layer applied to one token, and units
+// run strictly one after another (unit u+1 computes only after every output of unit u is
+// written; its weights may be fetched earlier). One CTA per SM. Every CTA owns a contiguous,
+// equal share of the rows of every phase of a unit:
+//   router rows      [E router rows, then the shared-gate vector as row E]  -> logits
+//   h-rows           I rows of every expert's gate and up matrices (the same rows for the
+//                    shared expert and for each routed expert)            -> h = SiLU(g) * u
+//   output rows      H rows of every expert's down matrix                  -> out
+// The share of each phase is cut into chunks of at most one shared-memory stage and streamed
+// through two rings of stages:
+//   ring A (data-independent weights, streamed ahead across units): the CTA's router chunks,
+//          shared-expert gate/up chunks and shared-expert down chunks of each unit;
+//   ring B (weights that depend on the routing decision): the routed experts' gate/up chunks
+//          (expert k = 0..K-1 in turn), then their down chunks.
+// The consumer warps work through a unit in the order
+//   router (A) -> shared gate/up (A) -> shared down (A) -> routed gate/up k (B) -> routed down k (B)
+// with every warp taking part in every chunk. Cross-CTA dependencies are counted on monotone
+// global counters (one per signal, each on its own 128-byte line): a CTA adds the number of
+// rows it finished; signal s of unit u is complete when its counter reaches (u + 1) times the
+// rows of that phase.
 #pragma once
 #include <stdint.h>
 
@@ -26,24 +27,25 @@ namespace fmoe {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kCtrlWarps = 2;                      // producer + stager
+constexpr int kCtrlWarps = 3;                      // producer A, producer B, controller
 constexpr int kThreads = kConsumers + 32 * kCtrlWarps;
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
-constexpr int kRowsPerLane = 8;                    // rows one lane accumulates per chunk
-constexpr int kStageTarget = 11520;                // bytes of weights per chunk (target)
-constexpr int kMaxStages = 32;
+constexpr unsigned kStage = 18432;                 // bytes per ring stage
+constexpr int kMaxStages = 16;                     // per ring
+constexpr int kMaxRowsThread = 8;                  // gate/up rows one consumer thread holds
+constexpr int kMaxRowsWarp = 8;                    // down rows (per side-by-side lane group) a warp holds
+constexpr int kMaxHr = 64;                         // h-rows per gate/up chunk (cap)
 
-enum Kind { K_ROUTER = 0, K_SGU = 1, K_RGU = 2, K_DN = 3, K_COUNT = 4 };
-enum Class { CL_ROUTER = 0, CL_GU = 1, CL_DN = 2, CL_COUNT = 3 };
-
-// Control words (uint32, zeroed before every launch). Class counters take one atomic per CTA
-// per run of same-class chunks; class c is complete for units 0..u when its counter reaches
-// (u + 1) * ncl[c], which the waiters (one warp per CTA) read directly.
-enum Ctrl {
-  C_CNT = 0,                    // C_CNT + 32*class: chunks of that class completed (all units)
-  C_WORDS = 32 * CL_COUNT       // every counter on its own 128-byte line
+// Global signals (counters in Scratch::ctrl, one 128-byte line each).
+enum Sig {
+  SG_ROUTER = 0,   // router rows finished (logits written)
+  SG_SHARED = 1,   // shared-expert h-rows finished
+  SG_OUT = 2,      // output rows finished (out written, sum of squares added)
+  SG_EXP0 = 3,     // + k: routed expert k's h-rows finished
+  SG_COUNT = SG_EXP0 + kMaxK
 };
+constexpr int kCtrlWords = 32 * SG_COUNT;
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
 
@@ -55,14 +57,6 @@ struct LayerW {
   const float* gate;           // nullable [H]
 };
 
-// Lane layout of a dot-product chunk inside one warp: S lanes share a row (S a power of two,
-// >= the row's 32-column slices when they are fewer than 32), P = 32 / S rows side by side.
-struct LaneMap {
-  int nsl;                     // 32-column slices per (virtual) row
-  int S, P;                    // lanes per row, rows side by side
-  int nrl;                     // rows per lane (<= kRowsPerLane)
-};
-
 struct Geo {
   int H, I, E, K, bits;
   int route_on, shared_on, routed_on, gate_on;
@@ -70,34 +64,38 @@ struct Geo {
   unsigned long long q_gu;          // bytes of one I x H packed matrix (gate or up)
   // router chunks
   int nr;                      // router rows: E + gate_on
-  int rseg;                    // column segments per router row
-  int rcols;                   // columns per segment (H / rseg)
-  int rrows;                   // router rows per chunk (1 when rseg > 1)
-  int nrb;                     // router row blocks: ceil(nr / rrows)
+  int rseg;                    // column segments per router row (1 when a row fits a stage)
+  int rcols;                   // columns per segment
+  int rrows;                   // router rows per chunk (rseg == 1)
   // gate/up chunks
-  int R;                       // rows of gate (and as many of up) per chunk
-  int nb;                      // chunks per expert: ceil(I / R)
+  int au;                      // h-row alignment unit (rows whose sb bytes are a multiple of 16)
+  int hr;                      // h-rows per chunk (a multiple of au)
   // down chunks
-  int nseg;                    // segments of a down virtual row: shared_on + K (routed)
-  int Rd;                      // virtual rows per chunk
-  int n[K_COUNT];
-  int off[K_COUNT + 1];        // off[K_COUNT] = chunks per unit
-  int ncl[CL_COUNT];           // chunks per unit of each class
-  LaneMap gu, dn;
+  int ad;                      // output-row alignment unit
+  int dr;                      // output rows per chunk (a multiple of ad)
+  int nseg;                    // down segments per output row: shared_on + K (routed)
+  // consumer thread layout for H-wide rows: slices S_h = H/32, W_h threads per row (a power
+  // of two >= S_h up to 32, else a multiple of 32), G_h = 256 / W_h row groups
+  int sh, wh, gh;
+  // consumer layout for I-wide rows: slices S_i = I/32; W_i lanes per row (power of two
+  // >= S_i, at most 32); P_i = 32 / W_i rows side by side in a warp; J_i slices per lane
+  int si, wi, pi, ji;
   // shared memory carve-up (byte offsets from the dynamic smem base)
   unsigned stage_bytes;
-  int nstage;
-  unsigned o_ring, o_full, o_empty, o_xa, o_xg, o_red, o_misc;
+  int nA, nB;                  // stages of ring A and ring B
+  unsigned o_ringA, o_ringB, o_x, o_h, o_red, o_oacc, o_misc, o_bar;
+  int oacc_n;                  // output accumulators (most output rows a CTA owns)
+  unsigned red_slot;           // bytes of the reduction area per stage (both rings)
   unsigned smem_bytes;
 };
 
 struct Scratch {
-  unsigned* ctrl;        // C_WORDS
+  unsigned* ctrl;        // kCtrlWords, zeroed per launch
   int* err;              // sticky per-device error word
-  double* logits;        // [2][rseg][nr] partial logits per column segment
+  double* logits;        // [2][rseg][nr] per unit parity: partial logits per column segment
   float* hs;             // [2][I]
   float* hk;             // [2][K][I]
-  float* normsq;         // [n_units]
+  float* normsq;         // [n_units], zeroed per launch
   float* hbuf;           // [2][H]
 };
 
@@ -112,14 +110,28 @@ struct Prog {
   float* w_out;          // SEQ: [T x K]; nullable
   float* h_trace;        // STACK: [T x L x H] layer inputs before the norm; nullable
   float eps;
+  int form;              // dot-product form (DotForm)
   unsigned long long wait_ns;
-  int debug;             // bit 0: the routing decision is never published (timeout test)
+  int debug;             // bit 0: the router signal is never raised (timeout test)
   Scratch s;
   LayerW layers[kMaxLayers];
 };
 
+// Evaluation of one group-affine dot product over a 32-column slice (same value in real
+// arithmetic): integer products of the codes with three 8-bit digit planes of x (default),
+// the pages' literal fma(q, s*x, z*x) per weight, or the naive (q*s + z)*x per weight.
+enum DotForm { FORM_DIGITS = 0, FORM_FMA = 1, FORM_NAIVE = 2, FORM_COUNT = 3 };
+
 // error codes written to Scratch::err (first one wins)
 enum DevErr { DE_NONE = 0, DE_TIMEOUT_FULL = 1, DE_TIMEOUT_EMPTY = 2, DE_TIMEOUT_ROUTE = 3,
               DE_TIMEOUT_DEP = 4, DE_TIMEOUT_DRAIN = 5 };
+
+// The contiguous share [lo, hi) of n items (in units of `unit` items) that CTA c of nc owns.
+__host__ __device__ __forceinline__ void share_of(int n, int unit, int c, int nc, int* lo,
+                                                  int* hi) {
+  const long long nu = n / unit;
+  *lo = (int)(nu * c / nc) * unit;
+  *hi = (int)(nu * (c + 1) / nc) * unit;
+}
 
 }  // namespace fmoe

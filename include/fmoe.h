@@ -231,18 +231,29 @@ int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const f
 int fmoe_stack_graph_launch(fmoe_graph* graph, void* stream);
 int fmoe_stack_graph_destroy(fmoe_graph* graph);
 
-/* Launch geometry of the engine kernel for a shape (host only; no CUDA call). flags: bit 0
- * router, bit 1 shared expert, bit 2 routed experts, bit 3 shared-expert gate. Writes up to
- * n_out int64 values in the order documented in FMOE_GEOMETRY_FIELDS and returns how many
- * were written, or a negative status for an unsupported shape. For checking the launch
- * layout against buffer bounds on a machine without a GPU. */
+/* Launch geometry of the engine kernel for a shape on a GPU with `sms` SMs and `max_smem`
+ * bytes of shared memory per block (host only; no CUDA call). flags: bit 0 router, bit 1
+ * shared expert, bit 2 routed experts, bit 3 shared-expert gate. Writes up to n_out int64
+ * values in the order documented in FMOE_GEOMETRY_FIELDS and returns how many were written,
+ * or a negative status for an unsupported shape. For checking the launch layout against
+ * buffer bounds on a machine without a GPU. */
 #define FMOE_GEOMETRY_FIELDS                                                                  \
     "H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr rseg rcols " \
-    "rrows nrb R nb nseg Rd n0 n1 n2 n3 off0 off1 off2 off3 off4 ncl0 ncl1 ncl2 gu_nsl gu_S "  \
-    "gu_P gu_nrl dn_nsl dn_S dn_P dn_nrl stage_bytes nstage o_ring o_full o_empty o_xa " \
-    "o_xg o_red o_misc smem_bytes"
+    "rrows au hr ad dr nseg sh wh gh si wi pi ji stage_bytes nA nB o_ringA o_ringB o_x o_h "    \
+    "o_red o_oacc o_misc o_bar oacc_n smem_bytes consumer_warps max_rows_thread max_rows_warp " \
+    "red_slot"
 int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int bits, int flags,
-                           int max_smem, int64_t* out, int n_out);
+                           int max_smem, int sms, int64_t* out, int n_out);
+
+/* Selects how the expert GEMVs evaluate each group-affine dot product, for kernels launched
+ * afterwards on the calling host thread (all give the same value in real arithmetic):
+ *   0  default: s * sum(q * x) + z * sum(x) per 32-column slice, sum(q * x) as integer dp4a
+ *      products of the codes with three signed 8-bit digit planes of x;
+ *   1  the pages' literal form per weight: sum of fma(q, s * x, z * x) ([FR-A] §2 "Noyaux de
+ *      Déquantification Optimisés pour FMA", the form after the rewrite);
+ *   2  the naive form per weight: sum of (q * s + z) * x ([FR-A] §2, the form before it).
+ * Returns FMOE_ERR_INVALID for another value (the setting is then unchanged). */
+int fmoe_set_dot_form(int form);
 
 /* Number of kernel launches of this library enqueued on the calling host thread so far
  * (graph replays count the kernels inside the graph). For accounting in benchmarks. */

@@ -1,7 +1,8 @@
-"""CPU check of the engine's launch geometry: every bulk copy the producer and the stager issue
-and every shared-memory read a consumer warp makes stays inside its buffer, its stage and the
-rows that were actually copied, for many shapes. Restates the address arithmetic of engine.cu
-on the host so that no out-of-range access is ever tried on a GPU first."""
+"""CPU check of the engine's launch geometry: every bulk copy the producers and the controller
+issue and every shared-memory access the consumer warps make stays inside its buffer, its stage
+and the rows that were actually copied, for many shapes and grid sizes; every router row,
+h-row and output row is owned by exactly one CTA. Restates the address arithmetic of
+engine.cu on the host, so that no out-of-range access is ever tried on a GPU first."""
 import itertools
 
 import pytest
@@ -9,216 +10,261 @@ import pytest
 fmoe = pytest.importorskip("bit_dequant_expert_gemv_b200")
 
 MAX_SMEM = 232448
-ROWS_PER_LANE = 8
-CONSUMER_WARPS = 8
+WARPS = 8
+THREADS = 256
 
 SHAPES = [
     # H, I, E, K, bits
     (4096, 1024, 512, 4, 4), (4096, 1024, 512, 4, 2), (256, 128, 16, 2, 4), (256, 128, 16, 2, 2),
     (64, 64, 1, 1, 4), (64, 64, 3, 3, 2), (192, 320, 7, 3, 4), (8192, 1024, 64, 8, 4),
     (7168, 2048, 256, 4, 4), (4160, 576, 33, 5, 2), (1024, 8192, 8, 1, 4), (2048, 704, 128, 6, 4),
-    (128, 64, 4096, 8, 2), (8128, 192, 16, 2, 4),
+    (128, 64, 4096, 8, 2), (8128, 192, 16, 2, 4), (128, 64, 1100, 8, 4), (1024, 576, 33, 5, 2),
+    (256, 128, 600, 4, 4), (8192, 8192, 2, 1, 2), (4608, 1024, 512, 4, 4),
 ]
 FLAGS = [15, 7, 5, 1, 2]  # full layer+gate, no gate, no shared, router only, expert only
-K_ROUTER, K_SGU, K_RGU, K_DN = range(4)
+GRIDS = [148, 132, 7, 1]
+CK_ROUTER, CK_GU, CK_DN = range(3)
 
 
-def chunks(G):
-    """(c, kind, j, k, seg, r0, n) for every chunk of one unit, as the kernel decodes them."""
-    for c in range(G["off4"]):
-        kind = max(i for i in range(4) if G[f"off{i}"] <= c and G[f"n{i}"] > 0)
-        j = c - G[f"off{kind}"]
-        k = seg = 0
-        if kind == K_ROUTER:
-            rb, seg = divmod(j, G["rseg"])
-            r0 = rb * G["rrows"]
-            n = min(G["rrows"], G["nr"] - r0)
-        elif kind == K_SGU:
-            r0, n = j * G["R"], min(G["R"], G["I"] - j * G["R"])
-        elif kind == K_RGU:
-            k, jj = divmod(j, G["nb"])
-            r0, n = jj * G["R"], min(G["R"], G["I"] - jj * G["R"])
-        else:
-            r0, n = j * G["Rd"], min(G["Rd"], G["H"] - j * G["Rd"])
-        assert n > 0
-        yield c, kind, j, k, seg, r0, n
+def share(n, unit, c, nc):
+    nu = n // unit
+    return (nu * c // nc) * unit, (nu * (c + 1) // nc) * unit
 
 
-def producer_copies(G, kind, k, seg, r0, n):
-    """(buffer, src_off, dst_off, bytes) per copy, as the producer issues them."""
+def make_share(G, c, nc):
+    S = {}
+    S["r0"], S["r1"] = share(G["nr"], 1, c, nc)
+    S["h0"], S["h1"] = share(G["I"], G["au"], c, nc)
+    S["d0"], S["d1"] = share(G["H"], G["ad"], c, nc)
+    nrr = S["r1"] - S["r0"]
+    if not G["route_on"]:
+        S["nrc"] = 0
+    elif G["rseg"] > 1:
+        S["nrc"] = nrr * G["rseg"]
+    else:
+        S["nrc"] = -(-nrr // G["rrows"])
+    gu = G["shared_on"] or G["routed_on"]
+    S["ngc"] = -(-(S["h1"] - S["h0"]) // G["hr"]) if gu else 0
+    S["ndc"] = -(-(S["d1"] - S["d0"]) // G["dr"]) if G["nseg"] > 0 else 0
+    S["na"] = S["nrc"] + (S["ngc"] + S["ndc"] if G["shared_on"] else 0)
+    S["nb"] = G["K"] * (S["ngc"] + S["ndc"]) if G["routed_on"] else 0
+    return S
+
+
+def chunk_a(G, S, i):
+    if i < S["nrc"]:
+        if G["rseg"] > 1:
+            rr, seg = divmod(i, G["rseg"])
+            return CK_ROUTER, -1, S["r0"] + rr, 1, seg
+        r0 = S["r0"] + i * G["rrows"]
+        return CK_ROUTER, -1, r0, min(G["rrows"], S["r1"] - r0), 0
+    i -= S["nrc"]
+    if i < S["ngc"]:
+        r0 = S["h0"] + i * G["hr"]
+        return CK_GU, -1, r0, min(G["hr"], S["h1"] - r0), 0
+    i -= S["ngc"]
+    r0 = S["d0"] + i * G["dr"]
+    return CK_DN, -1, r0, min(G["dr"], S["d1"] - r0), 0
+
+
+def chunk_b(G, S, i):
+    gu = G["K"] * S["ngc"]
+    if i < gu:
+        e, j = divmod(i, S["ngc"])
+        r0 = S["h0"] + j * G["hr"]
+        return CK_GU, e, r0, min(G["hr"], S["h1"] - r0), 0
+    i -= gu
+    e, j = divmod(i, S["ndc"])
+    r0 = S["d0"] + j * G["dr"]
+    return CK_DN, e, r0, min(G["dr"], S["d1"] - r0), 0
+
+
+def copies(G, kind, r0, n, seg):
+    """(buffer, src_off, dst_off, bytes) of each bulk copy, as copy_desc issues them."""
     H, I, E = G["H"], G["I"], G["E"]
     out = []
-    if kind == K_ROUTER:
-        if G["rseg"] == 1:
-            rowb = 4 * H
+    if kind == CK_ROUTER:
+        rowb = 4 * H
+        if G["rseg"] > 1:
+            buf, base = ("router", r0 * rowb) if r0 < E else ("gate", 0)
+            out.append((buf, base + seg * G["rcols"] * 4, 0, 4 * G["rcols"]))
+        else:
             a, b = r0, min(r0 + n, E)
             if b > a:
                 out.append(("router", a * rowb, 0, (b - a) * rowb))
             if r0 + n > E:
                 out.append(("gate", 0, (E - r0) * rowb, rowb))
-        else:
-            buf, base = ("router", r0 * 4 * H) if r0 < E else ("gate", 0)
-            out.append((buf, base + seg * G["rcols"] * 4, 0, 4 * G["rcols"]))
-    elif kind in (K_SGU, K_RGU):
-        buf = "shared" if kind == K_SGU else "expert"
-        cb, sbb = n * G["rc_h"], n * G["rs_h"]
-        sbo = I * G["rc_h"]
-        R = G["R"]
-        out += [(buf, r0 * G["rc_h"], 0, cb),
-                (buf, G["q_gu"] + r0 * G["rc_h"], R * G["rc_h"], cb),
-                (buf, sbo + r0 * G["rs_h"], 2 * R * G["rc_h"], sbb),
-                (buf, G["q_gu"] + sbo + r0 * G["rs_h"], 2 * R * G["rc_h"] + R * G["rs_h"], sbb)]
+    elif kind == CK_GU:
+        hr, rc, rs, q = G["hr"], G["rc_h"], G["rs_h"], G["q_gu"]
+        out += [("expert", r0 * rc, 0, n * rc), ("expert", q + r0 * rc, hr * rc, n * rc),
+                ("expert", I * rc + r0 * rs, 2 * hr * rc, n * rs),
+                ("expert", q + I * rc + r0 * rs, 2 * hr * rc + hr * rs, n * rs)]
     else:
-        cb, sbb = n * G["rc_i"], n * G["rs_i"]
-        Rd, nseg = G["Rd"], G["nseg"]
-        dsb = nseg * Rd * G["rc_i"]
-        dn = 2 * G["q_gu"]
-        for s in range(nseg):
-            buf = "shared" if (G["shared_on"] and s == 0) else "expert"
-            out += [(buf, dn + r0 * G["rc_i"], s * Rd * G["rc_i"], cb),
-                    (buf, dn + H * G["rc_i"] + r0 * G["rs_i"], dsb + s * Rd * G["rs_i"], sbb)]
+        dn, rc, rs = 2 * G["q_gu"], G["rc_i"], G["rs_i"]
+        out += [("expert", dn + r0 * rc, 0, n * rc),
+                ("expert", dn + H * rc + r0 * rs, G["dr"] * rc, n * rs)]
     return out
 
 
-def lane_reads(G, kind, n):
-    """Every shared-memory read of every lane of the consumer warp for a dot-product chunk:
-    yields (valid, code_off, code_bytes, sb_off, row, slice), including the clamped reads that
-    rows or slices outside the chunk make (valid False)."""
-    cbytes = 16 if G["bits"] == 4 else 8
-    if kind in (K_SGU, K_RGU):
-        pre = "gu"
-        nrows, R = 2 * G["R"], G["R"]
-        valid = lambda rho: rho < 2 * R and (rho if rho < R else rho - R) < n
-        rc, rs, seg_c, seg_s = G["rc_h"], G["rs_h"], 0, 0
-        sb0, spseg = 2 * R * G["rc_h"], G["H"] // 32
-    else:
-        pre = "dn"
-        nrows = n
-        valid = lambda rho: rho < n
-        rc, rs = G["rc_i"], G["rs_i"]
-        seg_c, seg_s = G["Rd"] * G["rc_i"], G["Rd"] * G["rs_i"]
-        sb0, spseg = G["nseg"] * G["Rd"] * G["rc_i"], G["I"] // 32
-    nsl, S, P, nrl = (G[f"{pre}_{f}"] for f in ("nsl", "S", "P", "nrl"))
-    NRL = 3 if nrl <= 3 else 4 if nrl == 4 else 6 if nrl <= 6 else 8
-    GW = 4 if NRL % 4 == 0 else 3
-    nj = (nsl + S - 1) // S
-    for lane in range(32):
-        ls, lp = lane % S, lane // S
-        for j in range(nj):
-            t = ls + S * j
-            tok = t < nsl
-            tc = t if tok else nsl - 1
-            seg, loc = divmod(tc, spseg)
-            cbase = seg * seg_c + loc * cbytes
-            sbase = sb0 + seg * seg_s + (loc >> 1) * 4
-            for g in range(0, NRL, GW):
-                if g and not P * g < nrows:
-                    continue
-                for w in range(GW):
-                    rho = lp + P * (g + w)
-                    ok = tok and valid(rho)
-                    rr = rho if ok else 0
-                    yield ok, cbase + rr * rc, cbytes, sbase + rr * rs, rho, tc
+def chunk_bytes(G, kind, n):
+    if kind == CK_ROUTER:
+        return 4 * G["rcols"] if G["rseg"] > 1 else 4 * G["H"] * n
+    if kind == CK_GU:
+        return 2 * n * (G["rc_h"] + G["rs_h"])
+    return n * (G["rc_i"] + G["rs_i"])
+
+
+def inside(cov, a, nb):
+    return any(lo <= a and a + nb <= hi for lo, hi in cov)
+
+
+def check_reads(G, kind, r0, n, seg, cov, NR, d0):
+    sb = G["stage_bytes"]
+    cb = 16 if G["bits"] == 4 else 8
+    if kind == CK_ROUTER:
+        cols = G["rcols"]
+        nf = cols // 4
+        assert nf <= 5 * THREADS  # the x columns a thread caches
+        for r in range(n):
+            for f in range(nf):
+                assert inside(cov, (r * nf + f) * 16, 16), (r, f)
+            assert (seg * cols + 4 * (nf - 1) + 4) <= G["H"]
+        assert (n * WARPS) * 8 <= G["red_slot"]
+        return
+    if kind == CK_GU:
+        hr, gh, wh, sh = G["hr"], G["gh"], G["wh"], G["sh"]
+        wn = wh // 32 if wh > 32 else 1
+        sb0 = 2 * hr * G["rc_h"]
+        for t in range(THREADS):
+            g, s = divmod(t, wh)
+            act = g < gh and s < sh
+            om = s >> 5 if wh > 32 else 0
+            for i in range(NR):
+                rho = g + gh * i
+                rr = rho if rho < hr else rho - hr
+                if act and rho < 2 * hr and rr < n:
+                    assert inside(cov, rho * G["rc_h"] + s * cb, cb), (t, rho, s)
+                    assert inside(cov, sb0 + rho * G["rs_h"] + (s >> 1) * 4, 4), (t, rho, s)
+                if act and rho < 2 * hr:
+                    assert (rho * wn + om) * 4 + 4 <= G["red_slot"]
+        # every valid row of the chunk is some thread's row
+        rows = {g + gh * i for g in range(gh) for i in range(NR)}
+        assert all(r in rows for r in range(n)) and all(hr + r in rows for r in range(n))
+        return
+    wi, pi, ji, si = G["wi"], G["pi"], G["ji"], G["si"]
+    sbb = G["dr"] * G["rc_i"]
+    seen = set()
+    for w in range(WARPS):
+        for lane in range(32):
+            ls, lp = lane % wi, lane // wi
+            for j in range(ji):
+                s = ls + wi * j
+                assert 32 * min(s, si - 1) + 32 <= G["I"]  # the slice's digit form
+                for i in range(NR):
+                    rho = w * pi + lp + WARPS * pi * i
+                    if s < si and rho < n:
+                        assert inside(cov, rho * G["rc_i"] + s * cb, cb), (w, lane, rho, s)
+                        assert inside(cov, sbb + rho * G["rs_i"] + (s >> 1) * 4, 4)
+                        seen.add(rho)
+                        assert r0 - d0 + rho < G["oacc_n"]
+    assert seen == set(range(n))
 
 
 @pytest.mark.parametrize("shape,flags", list(itertools.product(SHAPES, FLAGS)))
 def test_geometry_in_bounds(shape, flags):
     H, I, E, K, bits = shape
-    try:
-        G = fmoe.describe_geometry(H, I, E, K, bits, flags, MAX_SMEM)
-    except fmoe.FmoeError as e:
-        assert e.code == fmoe.FMOE_ERR_UNSUPPORTED
-        pytest.skip(str(e))
-    assert G["smem_bytes"] <= MAX_SMEM
-    ns, sb = G["nstage"], G["stage_bytes"]
-    assert 2 <= ns <= 32 and sb % 128 == 0
+    for nc in GRIDS:
+        try:
+            G = fmoe.describe_geometry(H, I, E, K, bits, flags, MAX_SMEM, nc)
+        except fmoe.FmoeError as e:
+            assert e.code == fmoe.FMOE_ERR_UNSUPPORTED
+            continue
+        check_geometry(G, nc)
+
+
+def check_geometry(G, nc):
+    H, I, E, K = G["H"], G["I"], G["E"], G["K"]
+    sb = G["stage_bytes"]
+    nA, nB = G["nA"], G["nB"]
+    assert G["smem_bytes"] <= MAX_SMEM and sb % 128 == 0
+    assert 1 <= nA <= 16 and 1 <= nB <= 16
     nseg = G["nseg"]
-    xa_len = 4 * max(H, nseg * I)
-    # carve-up: ring | fixed areas | barriers, non-overlapping and in order
-    # x areas: 128 bytes per 32-column slice (raw floats, or six digit chunks + {scale, sum})
-    areas = [("ring", 0, ns * sb), ("xa", G["o_xa"], xa_len), ("xg", G["o_xg"], 4 * H),
-             ("red", G["o_red"], 4 * CONSUMER_WARPS * 16 * ROWS_PER_LANE),
-             ("misc", G["o_misc"], 512), ("full", G["o_full"], 8 * ns), ("empty", G["o_empty"], 8 * ns)]
+    areas = [("ringA", G["o_ringA"], nA * sb), ("ringB", G["o_ringB"], nB * sb),
+             ("x", G["o_x"], 4 * H), ("h", G["o_h"], max(4 * nseg * I, 128)),
+             ("red", G["o_red"], G["red_slot"] * (nA + nB)), ("oacc", G["o_oacc"], 4 * max(G["oacc_n"], 1)),
+             ("misc", G["o_misc"], 512), ("bar", G["o_bar"], 16 * (nA + nB))]
     for (n1, a1, l1), (n2, a2, l2) in zip(areas, areas[1:]):
         assert a1 + l1 <= a2, (n1, n2)
     assert areas[-1][1] + areas[-1][2] <= G["smem_bytes"]
-    assert G["o_full"] % 8 == 0 and G["o_misc"] % 16 == 0
-    for name in ("o_xa", "o_xg", "o_red"):
-        assert G[name] % 16 == 0, name
-    # stager bulk copies into XA: x, then h_s | h_k
-    assert 4 * H <= xa_len and 4 * (nseg * I) <= xa_len
-    assert (4 * I) % 16 == 0 and (4 * K * I) % 16 == 0 and (4 * H) % 16 == 0
-    sizes = {"router": E * H * 4, "gate": H * 4, "shared": fmoe.expert_bytes(H, I, bits),
-             "expert": fmoe.expert_bytes(H, I, bits)}
+    for name, off, _ in areas[:-1]:
+        assert off % 128 == 0, name
+    assert G["o_bar"] % 8 == 0
+    # the controller's bulk copies: x (4H bytes), each h segment (4I bytes at 4I k)
+    assert (4 * H) % 16 == 0 and (4 * I) % 16 == 0
+    # consumer layouts
+    assert G["sh"] == H // 32 and G["gh"] * G["wh"] <= THREADS and G["gh"] >= 1
+    assert G["wh"] >= G["sh"] and (G["wh"] <= 32 or G["wh"] % 32 == 0)
+    if G["wh"] <= 32:
+        assert G["wh"] & (G["wh"] - 1) == 0
+    assert G["wi"] * G["pi"] == 32 and G["wi"] * G["ji"] >= G["si"]
+    nrg = -(-2 * G["hr"] // G["gh"])
+    nrd = -(-G["dr"] // (WARPS * G["pi"]))
+    assert max(nrg, nrd) <= 8
+    NR = 4 if max(nrg, nrd) <= 4 else 8
+    # transform work items stay inside their vectors
+    for bits_ts, nsl, length in [(4 if G["bits"] == 4 else 2, H // 32, H),
+                                 (4 if G["bits"] == 4 else 2, I // 32, I)]:
+        nv = 32 // bits_ts
+        assert nsl * 32 <= length and nv * bits_ts == 32
+    sizes = {"router": E * H * 4, "gate": H * 4,
+             "expert": fmoe.expert_bytes(H, I, G["bits"])}
     assert G["q_gu"] * 2 + H * (G["rc_i"] + G["rs_i"]) == sizes["expert"]
-    seen = set()
-    for c, kind, j, k, seg, r0, n in chunks(G):
-        copies = producer_copies(G, kind, k, seg, r0, n)
-        assert len(copies) <= 2 * 9
-        covered = []
-        for buf, so, do, nb in copies:
-            assert nb > 0 and nb % 16 == 0 and so % 16 == 0 and do % 16 == 0, (kind, buf, so, do, nb)
-            assert so + nb <= sizes[buf], (kind, buf, so, nb, sizes[buf])
-            assert do + nb <= sb, (kind, do, nb, sb)
-            covered.append((do, do + nb))
-        covered.sort()
-        for (a, b), (c2, d) in zip(covered, covered[1:]):
-            assert b <= c2, "copies overlap in the stage"
-        if kind == K_ROUTER:
-            # rows r0..r0+n-1 of rcols floats each, read as float4 by 32 lanes
-            assert n * 4 * G["rcols"] <= sb and G["rcols"] % 4 == 0
-            assert (seg + 1) * G["rcols"] <= H
-            assert sum(b - a for a, b in covered) == n * 4 * G["rcols"]
-            continue
-        if kind in (K_SGU, K_RGU):
-            assert r0 + n <= I and n <= G["R"] and k < K
-        else:
-            assert r0 + n <= H and n <= G["Rd"]
-        # lane reads: first, second and last (ragged) chunk of each kind
-        last = {K_SGU: G["nb"] - 1, K_RGU: G["nb"] - 1, K_DN: G["n3"] - 1}[kind]
-        jj = j % G["nb"] if kind == K_RGU else j
-        if jj not in (0, 1, last) or (kind, jj) in seen:
-            continue
-        seen.add((kind, jj))
-        pre = "gu" if kind in (K_SGU, K_RGU) else "dn"
-        x_len = H if pre == "gu" else nseg * I
-        assert G[f"{pre}_nrl"] <= ROWS_PER_LANE and G[f"{pre}_P"] <= 16
-        for ok, co, cbn, so, rho, t in lane_reads(G, kind, n):
-            assert 0 <= co and co + cbn <= sb and 0 <= so and so + 4 <= sb, (kind, co, so, sb)
-            assert 32 * t + 32 <= x_len, (kind, t, x_len)   # x' slice (the swizzle stays in it)
-            if ok:
-                assert any(a <= co and co + cbn <= b for a, b in covered), (kind, co, rho, t)
-                assert any(a <= so and so + 4 <= b for a, b in covered), (kind, so, rho, t)
-    # every output row and every h entry is produced exactly once per unit
-    ch = list(chunks(G))
-    if G["routed_on"] or G["shared_on"]:
-        assert sum(n for c, kd, j, k, s, r0, n in ch if kd == K_DN) == H
-        assert nseg == G["shared_on"] + (K if G["routed_on"] else 0)
-    if G["routed_on"]:
-        assert sum(n for c, kd, j, k, s, r0, n in ch if kd == K_RGU) == K * I
-    if G["shared_on"]:
-        assert sum(n for c, kd, j, k, s, r0, n in ch if kd == K_SGU) == I
-    if G["route_on"]:
-        assert sum(n for c, kd, j, k, s, r0, n in ch if kd == K_ROUTER) == G["nr"] * G["rseg"]
-    assert G["ncl0"] == G["n0"] and G["ncl1"] == G["n1"] + G["n2"] and G["ncl2"] == G["n3"]
+    own = {"r": [], "h": [], "d": []}
+    checked = set()  # the consumer reads depend only on (kind, valid rows, segment, row offset)
+    for c in range(nc):
+        S = make_share(G, c, nc)
+        own["r"].append((S["r0"], S["r1"]))
+        own["h"].append((S["h0"], S["h1"]))
+        own["d"].append((S["d0"], S["d1"]))
+        assert S["d1"] - S["d0"] <= max(G["oacc_n"], 0) or G["nseg"] == 0
+        lists = [chunk_a(G, S, i) for i in range(S["na"])] + [chunk_b(G, S, i) for i in range(S["nb"])]
+        covered_rows = {CK_ROUTER: [], CK_GU: {}, CK_DN: {}}
+        for kind, e, r0, n, seg in lists:
+            assert n > 0
+            cps = copies(G, kind, r0, n, seg)
+            cov = []
+            for buf, so, do, nb in cps:
+                assert nb > 0 and nb % 16 == 0 and so % 16 == 0 and do % 16 == 0, (kind, so, do, nb)
+                assert so + nb <= sizes[buf], (kind, buf, so, nb)
+                assert do + nb <= sb, (kind, do, nb, sb)
+                cov.append((do, do + nb))
+            cov.sort()
+            for (a, b), (c2, d) in zip(cov, cov[1:]):
+                assert b <= c2, "copies overlap in the stage"
+            assert sum(b - a for a, b in cov) == chunk_bytes(G, kind, n)
+            key = (kind, n, seg, r0 - S["d0"] if kind == CK_DN else 0)
+            if key not in checked:
+                checked.add(key)
+                check_reads(G, kind, r0, n, seg, cov, NR, S["d0"])
+            if kind == CK_ROUTER:
+                covered_rows[CK_ROUTER] += [(r, seg) for r in range(r0, r0 + n)]
+            else:
+                covered_rows[kind].setdefault(e, []).extend(range(r0, r0 + n))
+        if G["route_on"]:
+            assert sorted(covered_rows[CK_ROUTER]) == sorted(
+                (r, s) for r in range(S["r0"], S["r1"]) for s in range(G["rseg"]))
+        for kind, lo, hi in [(CK_GU, S["h0"], S["h1"]), (CK_DN, S["d0"], S["d1"])]:
+            for e, rows in covered_rows[kind].items():
+                assert sorted(rows) == list(range(lo, hi)), (kind, e)
+    # ownership: each phase's rows are split into disjoint contiguous shares covering all rows
+    for key, total in (("r", G["nr"]), ("h", I), ("d", H)):
+        spans = own[key]
+        assert spans[0][0] == 0 and spans[-1][1] == total
+        for (a, b), (c2, d) in zip(spans, spans[1:]):
+            assert b == c2 and a <= b
 
 
-def test_unsupported_shapes_are_refused():
-    for shape in [(16384, 1024, 8, 2, 4), (4096, 4096, 8, 4, 4), (4096, 1024, 16, 9, 4)]:
-        with pytest.raises(fmoe.FmoeError) as ei:
-            fmoe.describe_geometry(*shape)
-        assert ei.value.code == fmoe.FMOE_ERR_UNSUPPORTED
-    with pytest.raises(fmoe.FmoeError) as ei:
-        fmoe.describe_geometry(100, 128, 8, 2, 4)
-    assert ei.value.code == fmoe.FMOE_ERR_INVALID
-
-
-def test_full_shape_chunking():
-    """The 4-bit full-shape layer: 11.25 KB stages, gate/up chunks of 2+2 rows, down chunks of
-    4 virtual rows of 5 segments (so both run the same 4-row dot-product code), router rows
-    split in two column halves."""
-    G = fmoe.describe_geometry(4096, 1024, 512, 4, 4, 15, MAX_SMEM)
-    assert (G["rseg"], G["rcols"], G["R"], G["Rd"], G["nseg"]) == (2, 2048, 2, 4, 5)
-    assert G["stage_bytes"] == 11520 and G["nstage"] >= 16
-    assert (G["gu_S"], G["gu_P"], G["gu_nrl"]) == (32, 1, 4)
-    assert (G["dn_S"], G["dn_P"], G["dn_nrl"]) == (32, 1, 4)
+def test_main_shape_layout():
+    G = fmoe.describe_geometry(4096, 1024, 512, 4, 4, 15, MAX_SMEM, 148)
+    assert G["hr"] == 4 and G["nA"] >= 4 and G["nB"] >= 4 and G["oacc_n"] == 28
+    assert G["smem_bytes"] <= MAX_SMEM
