@@ -132,7 +132,7 @@ def expert_bytes(hidden: int, inter: int, bits: int) -> int:
 GEOMETRY_FIELDS = ("H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr "
                    "rseg rcols rrows au hr ad dr nseg sh wh gh si wi pi ji stage_bytes nA nB "
                    "o_ringA o_ringB o_x o_h o_red o_oacc o_misc o_bar oacc_n smem_bytes "
-                   "consumer_warps max_rows_thread max_rows_warp red_slot").split()
+                   "consumer_warps max_rows_thread max_rows_warp red_slot gpass").split()
 
 
 def describe_geometry(H, I, E, K, bits, flags=15, max_smem=232448, sms=148) -> dict:

@@ -145,7 +145,7 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   G->rc_h = (unsigned)H * bits / 8; G->rs_h = (unsigned)H / 16;
   G->rc_i = (unsigned)I * bits / 8; G->rs_i = (unsigned)I / 16;
   G->q_gu = (unsigned long long)I * (G->rc_h + G->rs_h);
-  if (sms < 1) return fail(FMOE_ERR_INVALID, "SM count %d", sms);
+  if (sms < 1 || sms > kMaxCtas) return fail(FMOE_ERR_UNSUPPORTED, "SM count %d", sms);
   const bool gu_on = shared_on || routed_on;
   G->nseg = (shared_on ? 1 : 0) + (routed_on ? K : 0);
   G->au = rows_for_16(G->rs_h);
@@ -156,14 +156,15 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
                 G->nseg > 0 ? (unsigned)G->ad * (G->rc_i + G->rs_i) : 0u}),
       128);
   G->stage_bytes = stage;
-  // router: whole rows when a row fits kStage bytes, else column segments of one row
+  // router: whole rows when a row fits kRouterCols columns, else column segments of one row
+  // (a consumer thread holds 4 float4 columns of a segment)
   G->nr = route_on ? E + (G->gate_on ? 1 : 0) : 0;
-  if (4u * H <= kStage) {
+  if (H <= kRouterCols) {
     G->rseg = 1;
     G->rcols = H;
     G->rrows = std::max(1, std::min(32, (int)(kStage / (4u * H))));
   } else {
-    int d = (int)((4u * H + kStage - 1) / kStage);
+    int d = (H + kRouterCols - 1) / kRouterCols;
     while (H % d || (H / d) % 4) ++d;
     G->rseg = d;
     G->rcols = H / d;
@@ -182,6 +183,8 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
     if (!gu_on) hr = G->au;  // no gate/up rows in this launch
     if (hr < G->au) return fail(FMOE_ERR_UNSUPPORTED, "gate/up rows do not fit a stage (H=%d)", H);
     G->hr = hr;
+    // two chunks in one pass when their rows fit the threads' row slots
+    G->gpass = (2 * 2 * hr <= kMaxRowsThread * G->gh) ? 2 : 1;
   }
   // down: lane layout, then dr output rows per chunk
   G->si = I / 32;
@@ -218,9 +221,9 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   const unsigned h_b = 4u * (unsigned)(G->nseg * I);
   const unsigned wn = G->wh > 32 ? (unsigned)G->wh / 32 : 1u;
   const unsigned red_slot = std::max(8u * (unsigned)G->rrows * kConsumerWarps,
-                                     4u * 2u * (unsigned)G->hr * wn);
+                                     4u * 2u * (unsigned)(G->gpass * G->hr) * wn);
   const unsigned oacc_b = 4u * (unsigned)std::max(G->oacc_n, 1);
-  const unsigned misc_b = 512;
+  const unsigned misc_b = kMiscBytes;
   const unsigned fixed = align_up(x_b, 128) + align_up(std::max(h_b, 128u), 128) +
                          align_up(oacc_b, 128) + misc_b;
   const unsigned per_stage = stage + red_slot + 16;
@@ -374,7 +377,7 @@ int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int 
                        G.rcols, G.rrows, G.au, G.hr, G.ad, G.dr, G.nseg, G.sh, G.wh, G.gh, G.si,
                        G.wi, G.pi, G.ji, G.stage_bytes, G.nA, G.nB, G.o_ringA, G.o_ringB, G.o_x,
                        G.o_h, G.o_red, G.o_oacc, G.o_misc, G.o_bar, G.oacc_n, G.smem_bytes,
-                       kConsumerWarps, kMaxRowsThread, kMaxRowsWarp, G.red_slot};
+                       kConsumerWarps, kMaxRowsThread, kMaxRowsWarp, G.red_slot, G.gpass};
   const int n = (int)(sizeof v / sizeof v[0]);
   for (int i = 0; i < n && i < n_out; ++i) out[i] = v[i];
   return n < n_out ? n : n_out;

@@ -41,7 +41,32 @@
 #include "engine.h"
 #include "ptx.cuh"
 
+// Timeline hooks (a point of a unit's progress reached by one role), used by an external
+// profiling build; they expand to nothing in the library.
+#ifndef FMOE_MARK
+#define FMOE_MARK(u, ev) ((void)0)
+#endif
+
 namespace fmoe {
+
+enum MarkEv {
+  MK_C_UNIT = 0, MK_C_PREV_DONE, MK_C_X, MK_C_S1, MK_C_RT, MK_C_XFREE, MK_C_SS, MK_C_HS,
+  MK_C_S2 = 8, MK_C_HK = 16,
+  MK_K_X = 24, MK_K_ROUTER, MK_K_XD, MK_K_SGU, MK_K_HS, MK_K_DS,
+  MK_K_P2F = 30, MK_K_P2 = 38, MK_K_HK = 46, MK_K_D = 54, MK_K_OUT = 62,
+  MK_B_RT = 63, MK_B_LAST, MK_A_FIRST, MK_A_LAST,
+  MK_R_DOT = 67, MK_R_RED, MK_R_LAST, MK_R_PUB,   // router batch: first and last consumer warp
+  MK_R_DOT_W = 71, MK_R_RED_W, MK_R_LAST_W,
+  MK_G_DOT = 74, MK_G_RED, MK_G_LAST, MK_G_PUB,   // first gate/up pass of routed expert 0
+  MK_G_DOT_W = 78, MK_G_RED_W, MK_G_LAST_W
+};
+// marks from the first (w == 0) and the last consumer warp inside a phase
+#define FMOE_MARK_W(u, ev0, evw)                                   \
+  do {                                                             \
+    const int w_ = ((int)threadIdx.x >> 5) - kCtrlWarps;           \
+    if (w_ == 0) FMOE_MARK(u, ev0);                                \
+    if (w_ == kConsumerWarps - 1) FMOE_MARK(u, evw);               \
+  } while (0)
 
 // ------------------------------------------------------------------------------------------
 // small shared state
@@ -64,76 +89,125 @@ struct Smem {
   float sigma[2];              // sigmoid(g . x) of the unit (1 without a shared gate)
   int rt_e[2][kMaxK];          // routing of unit u (index u & 1): experts and weights
   float rt_w[2][kMaxK];
+  // top-K candidates: each consumer warp's K best packed keys and their binary64 logits
+  unsigned long long cand_key[kConsumerWarps * kMaxK];
+  double cand_l[kConsumerWarps * kMaxK];
   volatile int abort;
 };
+static_assert(sizeof(Smem) <= kMiscBytes, "small shared state exceeds its area");
 
 __device__ __forceinline__ void raise_error(const Prog& P, Smem* sm, int code) {
   atomicCAS(P.s.err, 0, code);
   sm->abort = 1;
 }
 
-__device__ __forceinline__ unsigned* sig_word(const Prog& P, int s) { return P.s.ctrl + 32 * s; }
+__device__ __forceinline__ unsigned* sig_row(const Prog& P, int s) {
+  return P.s.ctrl + (size_t)s * kMaxCtas;
+}
+
+// This CTA has finished its rows of signal s for units 0..u (one lane; after every write of
+// those rows by this CTA is ordered before it, e.g. by a CTA barrier or an acquire chain).
+__device__ __forceinline__ void publish(const Prog& P, int s, int u) {
+  st_release(sig_row(P, s) + blockIdx.x, (unsigned)(u + 1));
+}
 
 // ------------------------------------------------------------------------------------------
 // bounded waits
 // ------------------------------------------------------------------------------------------
-// Spin until *a - target >= 0 (wrap-safe) on a gpu-scope counter, the budget runs out, the
-// CTA aborts or another CTA has recorded an error. Polls with relaxed loads and makes one
-// acquire fence once the target is seen.
-__device__ __noinline__ bool spin_geq(const Prog& P, Smem* sm, const unsigned* a, unsigned target,
-                                      int code) {
-  if ((int)(ld_acquire(a) - target) >= 0) return true;
-  const uint64_t deadline = global_ns() + P.wait_ns;
+// Whole warp: spin until every CTA's progress word of signal s has reached `target` (wrap-
+// safe), the budget runs out, the CTA aborts or another CTA has recorded an error. Lane l
+// polls words 4l..4l+3 and 128+4l.. with relaxed 16-byte loads; once every word is there,
+// every lane makes one acquire fence.
+__device__ __noinline__ bool warp_wait_sig(const Prog& P, Smem* sm, int s, unsigned target,
+                                           int code) {
+  const int lane = threadIdx.x & 31;
+  const int nc = gridDim.x;
+  const unsigned* row = sig_row(P, s);
+  uint64_t deadline = 0;
   for (unsigned it = 0;; ++it) {
-    if ((int)(ld_relaxed_gpu(a) - target) >= 0) {
+    bool ok = true;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int w0 = 4 * lane + 128 * h;
+      if (w0 < nc) {
+        const uint4 v = ld_relaxed_gpu_v4(row + w0);
+        ok = ok && (int)(v.x - target) >= 0;
+        ok = ok && (w0 + 1 >= nc || (int)(v.y - target) >= 0);
+        ok = ok && (w0 + 2 >= nc || (int)(v.z - target) >= 0);
+        ok = ok && (w0 + 3 >= nc || (int)(v.w - target) >= 0);
+      }
+    }
+    if (__all_sync(0xffffffffu, ok)) {
       fence_acq_rel_gpu();
       return true;
     }
-    if (sm->abort) return false;
-    if ((it & 15) == 15) {
-      if (ld_volatile_int(P.s.err) != 0) {
+    if (it == 0) deadline = global_ns() + P.wait_ns;
+    int bad = 0;
+    if (lane == 0 && (it & 7) == 7) {
+      if (sm->abort || ld_volatile_int(P.s.err) != 0) {
         sm->abort = 1;
-        return false;
-      }
-      if (global_ns() > deadline) {
+        bad = 1;
+      } else if (global_ns() > deadline) {
         raise_error(P, sm, code);
-        return false;
+        bad = 1;
       }
     }
-    __nanosleep(32);
+    if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+    __nanosleep(20);
   }
+}
+
+// Waits on shared-memory barriers and counters poll with short sleeps in between by default;
+// a positive FMOE_WAIT_SUSPEND_NS selects a try_wait that suspends the thread with that time
+// hint instead (the two measured the same).
+#ifndef FMOE_WAIT_SUSPEND_NS
+#define FMOE_WAIT_SUSPEND_NS 0
+#endif
+
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, unsigned parity) {
+  if (FMOE_WAIT_SUSPEND_NS > 0) return mbar_try_wait_sleep(bar, parity, FMOE_WAIT_SUSPEND_NS);
+  if (mbar_try_wait(bar, parity)) return true;
+  __nanosleep(20);
+  return false;
 }
 
 __device__ __noinline__ bool wait_mbar(const Prog& P, Smem* sm, uint64_t* bar, unsigned parity,
                                        int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
-  for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
-    if (sm->abort) return false;
-    if (global_ns() > deadline) {
-      raise_error(P, sm, code);
-      return false;
+  for (unsigned it = 0;; ++it) {
+    if (mbar_poll(bar, parity)) return true;
+    if ((it & 7) == 7) {
+      if (sm->abort) return false;
+      if (global_ns() > deadline) {
+        raise_error(P, sm, code);
+        return false;
+      }
     }
   }
 }
 
-// Wait until the readiness counter *cnt reaches target. Sleeps on the phase that the next
-// increment completes (the publisher stores the counter before it arrives on the barrier),
-// re-reading the counter after every wake-up or after at most ~1 us.
+// Wait until the readiness counter *cnt reaches target (the publisher stores the counter
+// with release semantics; it also arrives on `bar`, which the suspending form sleeps on).
 __device__ __noinline__ bool wait_ready(const Prog& P, Smem* sm, const unsigned* cnt,
                                         uint64_t* bar, unsigned target, int code) {
   unsigned c = ld_acquire_cta_smem(cnt);
   if ((int)(c - target) >= 0) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
-  for (;;) {
-    if (!mbar_try_wait_sleep(bar, c & 1u, 1000u)) __nanosleep(64);
+  for (unsigned it = 0;; ++it) {
+    if (FMOE_WAIT_SUSPEND_NS > 0) {
+      if (!mbar_try_wait_sleep(bar, c & 1u, FMOE_WAIT_SUSPEND_NS)) __nanosleep(64);
+    } else {
+      __nanosleep(20);
+    }
     c = ld_acquire_cta_smem(cnt);
     if ((int)(c - target) >= 0) return true;
-    if (sm->abort) return false;
-    if (global_ns() > deadline) {
-      raise_error(P, sm, code);
-      return false;
+    if ((it & 7) == 7) {
+      if (sm->abort) return false;
+      if (global_ns() > deadline) {
+        raise_error(P, sm, code);
+        return false;
+      }
     }
   }
 }
@@ -157,15 +231,6 @@ __device__ __forceinline__ bool warp_wait_mbar(const Prog& P, Smem* sm, uint64_t
                                                unsigned parity, int code) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = wait_mbar(P, sm, bar, parity, code);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool warp_spin_geq(const Prog& P, Smem* sm, int s, unsigned target,
-                                              int code) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = spin_geq(P, sm, sig_word(P, s), target, code);
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;
@@ -434,6 +499,8 @@ __device__ void producer_a(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
         failed = true;
         break;
       }
+      if (i == 0) FMOE_MARK(u, MK_A_FIRST);
+      if (i == S.na - 1) FMOE_MARK(u, MK_A_LAST);
       ++issued;
     }
   }
@@ -453,6 +520,7 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
       failed = true;
       break;
     }
+    FMOE_MARK(u, MK_B_RT);
     const int* rte = sm->rt_e[u & 1];
     for (int i = 0; i < S.nb; ++i) {
       const Chunk c = chunk_b(G, S, i);
@@ -464,6 +532,7 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
         failed = true;
         break;
       }
+      if (i == S.nb - 1) FMOE_MARK(u, MK_B_LAST);
       ++issued;
     }
   }
@@ -487,58 +556,7 @@ __device__ __forceinline__ unsigned long long pkey(double l, int e) {
   return (dkey(l) & ~0x1FFFull) | (unsigned long long)(0x1FFF - e);
 }
 
-__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
-  return a > b ? a : b;
-}
-
-// Sort 16 keys in descending order (bitonic network, fully unrolled).
-__device__ __forceinline__ void sort16_desc(unsigned long long (&k)[16]) {
-#pragma unroll
-  for (int size = 2; size <= 16; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long a = k[i], b = k[j];
-          const bool sw = desc ? (a < b) : (a > b);
-          k[i] = sw ? b : a;
-          k[j] = sw ? a : b;
-        }
-      }
-    }
-  }
-}
-
-// Logits e0 + lane + 32 i (i < 16) of the unit: the bias plus the column-segment partials,
-// in segment order.
-__device__ __forceinline__ void load_logits(const Geo& G, const double* lg, const float* bias,
-                                            int e0, double (&lv)[16]) {
-  const int lane = threadIdx.x & 31;
-  double p1[16];
-  float bv[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {  // the bias and the first two segments in one round trip
-    const int ec = min(e0 + lane + 32 * i, G.E - 1);
-    bv[i] = bias ? __ldcg(bias + ec) : 0.f;
-    lv[i] = __ldcg(lg + ec);
-    p1[i] = G.rseg > 1 ? __ldcg(lg + (size_t)G.nr + ec) : 0.0;
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) lv[i] = ((double)bv[i] + lv[i]) + p1[i];
-  for (int sg = 2; sg < G.rseg; ++sg) {
-    double part[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      part[i] = __ldcg(lg + (size_t)sg * G.nr + min(e0 + lane + 32 * i, G.E - 1));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) lv[i] += part[i];
-  }
-}
-
-// The binary64 logit of expert e (bias first, then the segments in order, as load_logits).
+// The binary64 logit of expert e: the bias first, then the column-segment partials in order.
 __device__ __forceinline__ double one_logit(const Geo& G, const double* lg, const float* bias,
                                             int e) {
   double l = ((double)(bias ? __ldcg(bias + e) : 0.f) + __ldcg(lg + e)) +
@@ -547,65 +565,114 @@ __device__ __forceinline__ double one_logit(const Geo& G, const double* lg, cons
   return l;
 }
 
-// Top-K of the unit's logits by one warp. Lane l holds experts l + 32 i of each block of 512;
-// with more than 512 experts every lane keeps its 16 largest keys across blocks (bitonic
-// merge). K rounds: the warp maximum of the lanes' best packed keys (two 32-bit reductions:
-// high word, then low word among the lanes holding that high word); the lane that held it
-// drops it. The winners' binary64 logits give the weights w_k = exp(l_k - l_max) /
-// sum_sel exp(l_j - l_max): the softmax over all experts followed by renormalisation over the
-// selected ones, where the full softmax denominator cancels.
-__device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int* rt_e,
-                          float* rt_w, int* idx_out, float* w_out) {
+// Top-K of the unit's logits by the consumer warps, after every CTA's router rows are in.
+// Warp w takes experts e = e0 + 32 w + lane + 32 W i (i = 0, 1; W consumer warps) of each
+// block of 64 W experts: their binary64 logits (bias first, then the column-segment partials
+// in order) and packed keys (pkey). Rounds of a warp maximum (two 32-bit reductions: high
+// word, then low word among the lanes holding it; the lane holding the winner drops it)
+// leave the warp's K best in lanes 0..K-1; further blocks' K best are merged into them the
+// same way. The warps' candidates go to shared memory; after a consumer barrier warp 0 merges
+// them and forms the weights w_k = exp(l_k - l_max) / sum_sel exp(l_j - l_max): the softmax
+// over all experts followed by renormalisation over the selected ones, where the full softmax
+// denominator cancels. Keys carry the index, so no two are equal; logits within ~2^-39
+// relative of each other count as tied and go to the lower index.
+
+// K rounds of a warp maximum over the M keys per lane; lane k < K ends with the k-th best key
+// and its logit (others: 0).
+template <int M>
+__device__ __forceinline__ void warp_topk(int K, unsigned long long (&key)[M], double (&lv)[M],
+                                          unsigned long long& out_key, double& out_l) {
   const int lane = threadIdx.x & 31;
-  unsigned long long key[16];
-  {
-    double lv[16];
-    load_logits(G, lg, bias, 0, lv);
+  out_key = 0ull;
+  out_l = 0.0;
+  for (int k = 0; k < K; ++k) {
+    unsigned long long bk = key[0];
+    int bi = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) key[i] = lane + 32 * i < G.E ? pkey(lv[i], lane + 32 * i) : 0ull;
-  }
-  if (G.E > 512) {
-    sort16_desc(key);
-    for (int e0 = 512; e0 < G.E; e0 += 512) {
-      double lw[16];
-      unsigned long long k2[16];
-      load_logits(G, lg, bias, e0, lw);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int e = e0 + lane + 32 * i;
-        k2[i] = e < G.E ? pkey(lw[i], e) : 0ull;
-      }
-      sort16_desc(k2);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) key[i] = umax64(key[i], k2[15 - i]);
-      sort16_desc(key);
-    }
-  }
-  unsigned long long bk = key[0];
-  int bi = 0;
-#pragma unroll
-  for (int i = 1; i < 16; ++i)
-    if (key[i] > bk) bk = key[i], bi = i;
-  int sel_e = 0;
-  for (int k = 0; k < G.K; ++k) {
+    for (int i = 1; i < M; ++i)
+      if (key[i] > bk) bk = key[i], bi = i;
     const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(bk >> 32));
     const unsigned lo =
         __reduce_max_sync(0xffffffffu, (unsigned)(bk >> 32) == hi ? (unsigned)bk : 0u);
     const unsigned long long win = ((unsigned long long)hi << 32) | lo;
-    if (bk == win && win != 0ull) {  // exactly one lane holds it: drop it, find the next
+    const bool mine = bk == win && win != 0ull;  // at most one lane holds it
+    double l = 0.0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) key[i] = i == bi ? 0ull : key[i];
-      bk = key[0];
-      bi = 0;
+    for (int i = 0; i < M; ++i) l = i == bi ? lv[i] : l;
+    const unsigned holder = __ballot_sync(0xffffffffu, mine);
+    const double wl = __shfl_sync(0xffffffffu, l, holder ? __ffs(holder) - 1 : 0);
+    if (mine) {
 #pragma unroll
-      for (int i = 1; i < 16; ++i)
-        if (key[i] > bk) bk = key[i], bi = i;
+      for (int i = 0; i < M; ++i) key[i] = i == bi ? 0ull : key[i];
     }
-    if (lane == k) sel_e = 0x1FFF - (int)(win & 0x1FFFull);
+    if (lane == k) {
+      out_key = win;
+      out_l = wl;
+    }
   }
+}
+
+__device__ __noinline__ void topk_block(const Prog& P, const Geo& G, Smem* sm, int u,
+                                        const double* lg, const float* bias, int* idx_out,
+                                        float* w_out) {
+  const int lane = threadIdx.x & 31;
+  const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
+  float gate_l = 0.f;
+  if (w == 0 && lane == 0 && G.gate_on) {  // the shared-gate row's logit (sigma), early
+    double a = 0.0;
+    for (int sg = 0; sg < G.rseg; ++sg) a += __ldcg(lg + (size_t)sg * G.nr + G.E);
+    gate_l = (float)a;
+  }
+  unsigned long long best_key = 0ull;  // lane k < K: the warp's k-th best so far
+  double best_l = 0.0;
+  constexpr int kBlock = 64 * kConsumerWarps;
+  for (int e0 = 0; e0 < G.E; e0 += kBlock) {
+    unsigned long long key[2];
+    double lv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int e = e0 + 32 * w + lane + 32 * kConsumerWarps * i;
+      lv[i] = one_logit(G, lg, bias, min(e, G.E - 1));
+      key[i] = e < G.E ? pkey(lv[i], e) : 0ull;
+    }
+    unsigned long long bk;
+    double bl;
+    warp_topk<2>(G.K, key, lv, bk, bl);
+    if (e0 == 0) {
+      best_key = bk;
+      best_l = bl;
+    } else {  // merge the block's K best (lanes 0..K-1) into the running K best
+      key[0] = best_key;
+      lv[0] = best_l;
+      key[1] = bk;
+      lv[1] = bl;
+      warp_topk<2>(G.K, key, lv, best_key, best_l);
+    }
+  }
+  if (lane < G.K) {
+    sm->cand_key[w * kMaxK + lane] = best_key;
+    sm->cand_l[w * kMaxK + lane] = best_l;
+  }
+  consumers_sync();
+  if (w != 0) return;
+  // merge: lane l holds candidates l + 32 i of the W K (missing ones are 0)
+  constexpr int kM = (kConsumerWarps * kMaxK + 31) / 32;
+  const int nc = kConsumerWarps * G.K;
+  unsigned long long key[kM];
+  double lv[kM];
+#pragma unroll
+  for (int i = 0; i < kM; ++i) {
+    const int c = lane + 32 * i;
+    const int wk = c / G.K, kk = c - wk * G.K;  // candidate kk of warp wk
+    const bool ok = c < nc;
+    key[i] = ok ? sm->cand_key[wk * kMaxK + kk] : 0ull;
+    lv[i] = ok ? sm->cand_l[wk * kMaxK + kk] : 0.0;
+  }
+  unsigned long long sel_key;
+  double sel_l;
+  warp_topk<kM>(G.K, key, lv, sel_key, sel_l);
   const bool mine = lane < G.K;
-  const int e = min(max(sel_e, 0), G.E - 1);  // NaN logits must not make an address
-  const double sel_l = mine ? one_logit(G, lg, bias, e) : 0.0;
+  const int e = min(max(0x1FFF - (int)(sel_key & 0x1FFFull), 0), G.E - 1);
   const double l0 = __shfl_sync(0xffffffffu, sel_l, 0);
   const float ex = mine ? expf((float)(sel_l - l0)) : 0.f;
   float den = ex;
@@ -613,12 +680,14 @@ __device__ void topk_warp(const Geo& G, const double* lg, const float* bias, int
   for (int o = 1; o < 32; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   if (mine) {
     const float wk = __fdividef(ex, den);
-    rt_e[lane] = e;
-    rt_w[lane] = wk;
+    sm->rt_e[u & 1][lane] = e;
+    sm->rt_w[u & 1][lane] = wk;
     if (idx_out) idx_out[lane] = e;
     if (w_out) w_out[lane] = wk;
   }
+  if (lane == 0) sm->sigma[u & 1] = G.gate_on ? 1.f / (1.f + expf(-gate_l)) : 1.f;
   __syncwarp();
+  if (lane == 0) signal_ready(&sm->rt_ready, &sm->rt_bar, (unsigned)(u + 1));
 }
 
 // ------------------------------------------------------------------------------------------
@@ -645,9 +714,6 @@ __device__ __forceinline__ bool wait_copy(const Prog& P, Smem* sm, uint64_t* bar
 
 // The signal whose completion means "unit u is done" and its rows per unit.
 __device__ __forceinline__ int final_sig(const Geo& G) { return G.nseg > 0 ? SG_OUT : SG_ROUTER; }
-__device__ __forceinline__ unsigned final_rows(const Geo& G) {
-  return G.nseg > 0 ? (unsigned)G.H : (unsigned)(G.nr * G.rseg);
-}
 
 __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
   const int lane = threadIdx.x & 31;
@@ -656,65 +722,48 @@ __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm)
   unsigned px = 0, ph = 0;  // phases of the x and h copy barriers
   bool x_issued = false;    // the next unit's x copy is already in flight
   const int fsig = final_sig(G);
-  const unsigned frows = final_rows(G);
-  bool x_digits = G.shared_on || G.routed_on;
+  const bool x_digits = G.shared_on || G.routed_on;
   for (int u = 0; u < P.n_units; ++u) {
     const UnitView uv = unit_view(P, G, u);
     const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
+    FMOE_MARK(u, MK_C_UNIT);
     // ---- x(u): computed on only after unit u-1 is complete everywhere
-    if (u > 0 && !warp_spin_geq(P, sm, fsig, (unsigned)u * frows, DE_TIMEOUT_DEP)) break;
+    if (u > 0 && !warp_wait_sig(P, sm, fsig, (unsigned)u, DE_TIMEOUT_DEP)) break;
+    FMOE_MARK(u, MK_C_PREV_DONE);
     if (!x_issued) copy_in(XB, uv.xin, 4u * (unsigned)G.H, &sm->xbar);
     x_issued = false;
     float f = 1.f;
     if (uv.norm) f = rsqrtf(__ldcg(P.s.normsq + (u - 1)) / (float)G.H + P.eps);
     if (!wait_copy(P, sm, &sm->xbar, px)) break;
+    FMOE_MARK(u, MK_C_X);
     if (owner && uv.h_trace)
       for (int c = lane * 4; c < G.H; c += 128)
         *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XB + c);
     if (lane == 0) {
       sm->xf[u & 1] = f;
+      if (!G.route_on) sm->sigma[u & 1] = 1.f;
       signal_ready(&sm->x_ready, &sm->x_bar, (unsigned)(u + 1));
     }
     __syncwarp();
-    // ---- routing decision: needs every router row of unit u
-    const double* lg = P.s.logits + (size_t)uv.slot * G.rseg * G.nr;
-    if (G.route_on) {
-      if (uv.bias)  // the unit's logit bias into L2 while the router runs
-        for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
-      if (!warp_spin_geq(P, sm, SG_ROUTER, (unsigned)(u + 1) * (unsigned)(G.nr * G.rseg),
-                         DE_TIMEOUT_ROUTE))
-        break;
-      topk_warp(G, lg, uv.bias, sm->rt_e[u & 1], sm->rt_w[u & 1], owner ? uv.idx_out : nullptr,
-                owner ? uv.w_out : nullptr);
-      float sigma = 1.f;
-      if (G.gate_on) {
-        double a = 0.0;
-        for (int s = 0; s < G.rseg; ++s) a += __ldcg(lg + (size_t)s * G.nr + G.E);
-        sigma = (float)(1.0 / (1.0 + exp(-a)));
-      }
-      if (lane == 0) {
-        sm->sigma[u & 1] = sigma;
-        signal_ready(&sm->rt_ready, &sm->rt_bar, (unsigned)(u + 1));
-      }
-      __syncwarp();
-    } else if (lane == 0) {
-      sm->sigma[u & 1] = 1.f;
-    }
+    if (G.route_on && uv.bias)  // the unit's logit bias into L2 while the router runs
+      for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
     // ---- independent tokens: the next unit's x, once the consumers hold this unit's x
     // digits in registers (its computation still waits for this unit to complete)
     if (P.mode == MODE_SEQ && x_digits && u + 1 < P.n_units) {
       if (!warp_wait_ready(P, sm, &sm->xfree, &sm->xfree_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
         break;
+      FMOE_MARK(u, MK_C_XFREE);
       copy_in(XB, P.x + (size_t)(u + 1) * G.H, 4u * (unsigned)G.H, &sm->xbar);
       x_issued = true;
     }
     if (G.nseg == 0) continue;
     // ---- h_s: every shared-expert h-row of unit u
     if (G.shared_on) {
-      if (!warp_spin_geq(P, sm, SG_SHARED, (unsigned)(u + 1) * (unsigned)G.I, DE_TIMEOUT_DEP))
-        break;
+      if (!warp_wait_sig(P, sm, SG_SHARED, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
+      FMOE_MARK(u, MK_C_SS);
       copy_in(HB, P.s.hs + (size_t)uv.slot * G.I, 4u * (unsigned)G.I, &sm->hbar);
       if (!wait_copy(P, sm, &sm->hbar, ph)) break;
+      FMOE_MARK(u, MK_C_HS);
       if (lane == 0) signal_ready(&sm->hs_ready, &sm->hs_bar, (unsigned)(u + 1));
       __syncwarp();
     }
@@ -722,12 +771,14 @@ __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm)
     if (G.routed_on) {
       bool ok = true;
       for (int k = 0; k < G.K && ok; ++k) {
-        ok = warp_spin_geq(P, sm, SG_EXP0 + k, (unsigned)(u + 1) * (unsigned)G.I, DE_TIMEOUT_DEP);
+        ok = warp_wait_sig(P, sm, SG_EXP0 + k, (unsigned)(u + 1), DE_TIMEOUT_DEP);
         if (!ok) break;
+        FMOE_MARK(u, MK_C_S2 + k);
         copy_in(HB + (size_t)(G.shared_on + k) * G.I, P.s.hk + ((size_t)uv.slot * G.K + k) * G.I,
                 4u * (unsigned)G.I, &sm->hbar);
         ok = wait_copy(P, sm, &sm->hbar, ph);
         if (!ok) break;
+        FMOE_MARK(u, MK_C_HK + k);
         if (lane == 0) signal_ready(&sm->hk_ready, &sm->hk_bar, (unsigned)(u * G.K + k + 1));
         __syncwarp();
       }
@@ -778,79 +829,53 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
                      __byte_perm((uint32_t)c, (uint32_t)d, 0x0040), 0x5410);
 }
 
+// Column of byte b (b = 0..3) of digit word n of a slice (see the layout above).
+template <int BITS>
+__device__ __forceinline__ int word_col(int n, int b) {
+  return BITS == 4 ? 8 * (n >> 1) + 2 * b + (n & 1) : 16 * (n >> 2) + 4 * b + (n & 3);
+}
+
 // Transform nsl slices of buf (binary32, scaled by `scale`) into digit form, in place, by the
-// 256 consumer threads: TS threads per slice, each owning one code word's columns (8 at
-// 4 bits, 16 at 2 bits). Every lane of a warp reads its values before any lane writes (the
-// TS threads of a slice are consecutive lanes of one warp).
+// 256 consumer threads: 8 threads per slice, thread n of a slice making digit word n of the
+// three planes from its four columns. The 8 threads of a slice are consecutive lanes of one
+// warp, and every lane reads its values before any lane writes.
 template <int BITS>
 __device__ void transform(float* buf, int nsl, float scale) {
-  constexpr int TS = BITS == 4 ? 4 : 2;
-  constexpr int NV = 32 / TS;
   const int t = (int)threadIdx.x - 32 * kCtrlWarps;
-  const int items = nsl * TS;
+  const int items = nsl * 8;
   const int rounds = (items + kConsumers - 1) / kConsumers;
+  uint32_t* base = reinterpret_cast<uint32_t*>(buf);
   for (int r = 0; r < rounds; ++r) {
     const int it = t + kConsumers * r;
     const bool act = it < items;
-    const int s = act ? it / TS : 0, j = it % TS;
-    float v[NV];
+    const int s = act ? it >> 3 : 0, n = it & 7;
+    float v[4];
     float m = 0.f, sum = 0.f;
-    if (act) {
 #pragma unroll
-      for (int q = 0; q < NV / 4; ++q) {
-        const float4 a = *reinterpret_cast<const float4*>(buf + 32 * s + NV * j + 4 * q);
-        v[4 * q] = a.x * scale; v[4 * q + 1] = a.y * scale;
-        v[4 * q + 2] = a.z * scale; v[4 * q + 3] = a.w * scale;
-      }
-#pragma unroll
-      for (int q = 0; q < NV; ++q) {
-        m = fmaxf(m, fabsf(v[q]));
-        sum += v[q];
-      }
+    for (int b = 0; b < 4; ++b) {
+      v[b] = act ? buf[32 * s + word_col<BITS>(n, b)] * scale : 0.f;
+      m = fmaxf(m, fabsf(v[b]));
     }
+    sum = (v[0] + v[1]) + (v[2] + v[3]);
 #pragma unroll
-    for (int o = 1; o < TS; o <<= 1) {
+    for (int o = 1; o < 8; o <<= 1) {
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       sum += __shfl_xor_sync(0xffffffffu, sum, o);
     }
     __syncwarp();
     if (act) {
-      const float k = m > 0.f ? __fdividef(2080768.f, m) : 0.f;
-      uint32_t* base = reinterpret_cast<uint32_t*>(buf);
-      if (BITS == 4) {
-        uint32_t w[3][2];
+      // the in-place factor of word n: 1 / 16 for high nibbles, 4^-p for bit-pair p
+      const float fw = BITS == 4 ? ((n & 1) ? 0.0625f : 1.f)
+                                 : ((n & 3) == 0 ? 1.f : (n & 3) == 1 ? 0.25f
+                                                       : (n & 3) == 2 ? 0.0625f : 0.015625f);
+      const float k = m > 0.f ? __fdividef(2080768.f, m) * fw : 0.f;
+      int d[3][4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float kh = h ? k * 0.0625f : k;
-          int d[3][4];
+      for (int b = 0; b < 4; ++b) digits3(v[b], k, d[0][b], d[1][b], d[2][b]);
 #pragma unroll
-          for (int b = 0; b < 4; ++b) digits3(v[2 * b + h], kh, d[0][b], d[1][b], d[2][b]);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) w[p][h] = pack4(d[p][0], d[p][1], d[p][2], d[p][3]);
-        }
-        // words 2j, 2j+1 of plane p: chunk 2p + j/2, word positions 2(j%2), 2(j%2)+1
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-          *reinterpret_cast<uint2*>(base + dslot(s, 2 * p + (j >> 1)) + 2 * (j & 1)) =
-              make_uint2(w[p][0], w[p][1]);
-      } else {
-        uint32_t w[3][4];
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          const float kp = k * (pc == 0 ? 1.f : pc == 1 ? 0.25f : pc == 2 ? 0.0625f : 0.015625f);
-          int d[3][4];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) digits3(v[4 * b + pc], kp, d[0][b], d[1][b], d[2][b]);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) w[p][pc] = pack4(d[p][0], d[p][1], d[p][2], d[p][3]);
-        }
-        // words 4j .. 4j+3 of plane p: chunk 2p + j
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-          *reinterpret_cast<uint4*>(base + dslot(s, 2 * p + j)) =
-              make_uint4(w[p][0], w[p][1], w[p][2], w[p][3]);
-      }
-      if (j == 0)
+      for (int p = 0; p < 3; ++p)
+        base[dslot(s, 2 * p + (n >> 2)) + (n & 3)] = pack4(d[p][0], d[p][1], d[p][2], d[p][3]);
+      if (n == 0)
         *reinterpret_cast<float2*>(base + dslot(s, 6)) = make_float2(m * (1.f / 2080768.f), sum);
     }
     __syncwarp();
@@ -864,16 +889,15 @@ struct XDig {
 };
 
 __device__ __forceinline__ void load_digits(const float* buf, int s, XDig& x) {
-  const uint32_t base = smem_u32(buf);
 #pragma unroll
   for (int i = 0; i < 6; ++i) {
-    const uint4 a = lds128(base + 4u * (unsigned)dslot(s, i));
+    const uint4 a = *reinterpret_cast<const uint4*>(buf + dslot(s, i));
     x.d[4 * i] = (int)a.x; x.d[4 * i + 1] = (int)a.y; x.d[4 * i + 2] = (int)a.z;
     x.d[4 * i + 3] = (int)a.w;
   }
-  const uint2 b = lds64(base + 4u * (unsigned)dslot(s, 6));
-  x.sc = __uint_as_float(b.x);
-  x.sx = __uint_as_float(b.y);
+  const float2 b = *reinterpret_cast<const float2*>(buf + dslot(s, 6));
+  x.sc = b.x;
+  x.sx = b.y;
 }
 
 // The binary32 values of slice s of buf, scaled (the literal and naive forms).
@@ -901,10 +925,10 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
 
 // s * sum(q x) + z * sum(x) over the slice: codes at `ca`, scale/bias word `sbw`.
 template <int BITS>
-__device__ __forceinline__ float slice_dot(uint32_t ca, uint32_t sbw, const XDig& x) {
+__device__ __forceinline__ float slice_dot(const uint8_t* ca, uint32_t sbw, const XDig& x) {
   int c0 = 0, c1 = 0, c2 = 0;
   if constexpr (BITS == 4) {
-    const uint4 q = lds128(ca);
+    const uint4 q = *reinterpret_cast<const uint4*>(ca);
     const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -914,7 +938,7 @@ __device__ __forceinline__ float slice_dot(uint32_t ca, uint32_t sbw, const XDig
       c2 = dp4a_us(hi, x.d[16 + 2 * j + 1], dp4a_us(lo, x.d[16 + 2 * j], c2));
     }
   } else {
-    const uint2 q = lds64(ca);
+    const uint2 q = *reinterpret_cast<const uint2*>(ca);
     const uint32_t qw[2] = {q.x, q.y};
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -942,13 +966,13 @@ __device__ __forceinline__ float code_at(const uint32_t* qw, int c) {
 
 // The pages' literal FMA form per weight: sum over the slice of fma(q, s*x, z*x).
 template <int BITS>
-__device__ __forceinline__ float slice_dot_fma(uint32_t ca, uint32_t sbw, const XVal& x) {
+__device__ __forceinline__ float slice_dot_fma(const uint8_t* ca, uint32_t sbw, const XVal& x) {
   uint32_t qw[4];
   if constexpr (BITS == 4) {
-    const uint4 q = lds128(ca);
+    const uint4 q = *reinterpret_cast<const uint4*>(ca);
     qw[0] = q.x; qw[1] = q.y; qw[2] = q.z; qw[3] = q.w;
   } else {
-    const uint2 q = lds64(ca);
+    const uint2 q = *reinterpret_cast<const uint2*>(ca);
     qw[0] = q.x; qw[1] = q.y; qw[2] = 0u; qw[3] = 0u;
   }
   const float s = __uint_as_float(sbw << 16);
@@ -964,13 +988,13 @@ __device__ __forceinline__ float slice_dot_fma(uint32_t ca, uint32_t sbw, const 
 
 // The naive form per weight: sum over the slice of (q*s + z) * x.
 template <int BITS>
-__device__ __forceinline__ float slice_dot_naive(uint32_t ca, uint32_t sbw, const XVal& x) {
+__device__ __forceinline__ float slice_dot_naive(const uint8_t* ca, uint32_t sbw, const XVal& x) {
   uint32_t qw[4];
   if constexpr (BITS == 4) {
-    const uint4 q = lds128(ca);
+    const uint4 q = *reinterpret_cast<const uint4*>(ca);
     qw[0] = q.x; qw[1] = q.y; qw[2] = q.z; qw[3] = q.w;
   } else {
-    const uint2 q = lds64(ca);
+    const uint2 q = *reinterpret_cast<const uint2*>(ca);
     qw[0] = q.x; qw[1] = q.y; qw[2] = 0u; qw[3] = 0u;
   }
   const float s = __uint_as_float(sbw << 16);
@@ -985,7 +1009,7 @@ __device__ __forceinline__ float slice_dot_naive(uint32_t ca, uint32_t sbw, cons
 }
 
 template <int BITS, int FORM, typename XT>
-__device__ __forceinline__ float slice_any(uint32_t ca, uint32_t sbw, const XT& x) {
+__device__ __forceinline__ float slice_any(const uint8_t* ca, uint32_t sbw, const XT& x) {
   if constexpr (FORM == FORM_DIGITS)
     return slice_dot<BITS>(ca, sbw, x);
   else if constexpr (FORM == FORM_FMA)
@@ -1009,9 +1033,8 @@ struct XOf<FORM_DIGITS> {
 // Transposing butterfly over `width` lanes (a power of two <= 32, the lane's segment): NR row
 // partials per lane become one fully reduced value per row; store(i, v) is called for row i
 // on exactly one lane of the segment.
-template <int NR, typename Store>
-__device__ __forceinline__ void seg_reduce(float (&v)[NR], int lane_in_seg, int width,
-                                           Store store) {
+template <int NR, typename T, typename Store>
+__device__ __forceinline__ void seg_reduce(T (&v)[NR], int lane_in_seg, int width, Store store) {
   int lo = 0;
   int nlive = NR;
 #pragma unroll
@@ -1023,8 +1046,8 @@ __device__ __forceinline__ void seg_reduce(float (&v)[NR], int lane_in_seg, int 
 #pragma unroll
       for (int a = 0; a < (NR >> 1); ++a) {
         if (a < half) {
-          const float send = upper ? v[a] : v[a + half];
-          const float keep = upper ? v[a + half] : v[a];
+          const T send = upper ? v[a] : v[a + half];
+          const T keep = upper ? v[a + half] : v[a];
           v[a] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
       }
@@ -1045,14 +1068,32 @@ __device__ __forceinline__ void seg_reduce(float (&v)[NR], int lane_in_seg, int 
 // ------------------------------------------------------------------------------------------
 // consumer warps
 // ------------------------------------------------------------------------------------------
+// A ring of stages (ring A or ring B); the consumers' count of chunks taken from each ring is
+// kept in registers beside it. Copied by value (never addressed) so that it stays in registers.
 struct Ring {
   uint8_t* base;
   uint64_t* full;
   uint64_t* empty;
   int ns;
   int slot0;       // first chunk_arrive / red slot of this ring
-  unsigned used;   // chunks consumed so far
 };
+
+__device__ __forceinline__ const uint8_t* ring_stage(const Geo& G, const Ring& R, unsigned use) {
+  return R.base + (size_t)(use % (unsigned)R.ns) * G.stage_bytes;
+}
+__device__ __forceinline__ uint64_t* ring_empty(const Ring& R, unsigned use) {
+  return &R.empty[use % (unsigned)R.ns];
+}
+__device__ __forceinline__ int ring_slot(const Ring& R, unsigned use) {
+  return R.slot0 + (int)(use % (unsigned)R.ns);
+}
+// Wait (whole warp) for chunk `use` of the ring to have landed.
+__device__ __forceinline__ void ring_wait(const Prog& P, Smem* sm, const Ring& R, unsigned use,
+                                          bool& dead) {
+  if (!dead && !warp_wait_mbar(P, sm, &R.full[use % (unsigned)R.ns], (use / (unsigned)R.ns) & 1u,
+                               DE_TIMEOUT_FULL))
+    dead = true;
+}
 
 // Every warp arrives once per chunk use of a stage; the warp that completes the count of 8
 // returns true (it has acquired every other warp's writes of the chunk) and resets it.
@@ -1076,8 +1117,9 @@ __device__ __forceinline__ void release_stage(uint64_t* empty) {
 // Router rows of a chunk: binary64 sums of fp32 products over the chunk's columns; each
 // thread takes float4 columns t, t + 256, ...; per row a warp reduction, the 8 warp
 // partials through shared memory, summed in warp order by the chunk's last warp.
+// This thread's x columns (float4 t + 512 j, j < 4) of the router segment it last loaded.
 struct XRouter {
-  double v[5][4];   // this thread's x columns (binary64) of the current segment
+  float4 v[4];
   int seg;          // which segment they hold (-1: none)
 };
 
@@ -1086,14 +1128,72 @@ __device__ __forceinline__ void router_x(const Geo& G, const float* XB, int seg,
   const int nf = G.rcols / 4;
   const float4* xs = reinterpret_cast<const float4*>(XB + (size_t)seg * G.rcols);
 #pragma unroll
-  for (int j = 0; j < 5; ++j) {
+  for (int j = 0; j < 4; ++j) {
     const int f = t + kConsumers * j;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (f < nf) a = xs[f];
-    xr.v[j][0] = (double)a.x; xr.v[j][1] = (double)a.y;
-    xr.v[j][2] = (double)a.z; xr.v[j][3] = (double)a.w;
+    xr.v[j] = f < nf ? xs[f] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   xr.seg = seg;
+}
+
+// sum over the float4 columns of one row: four products each, converted to binary64 (exact)
+// and accumulated in binary64
+__device__ __forceinline__ double row_dot4(const float4* ws, int f, const float4& x) {
+  const float4 wv = ws[f];
+  double a = (double)wv.x * (double)x.x;
+  a = fma((double)wv.y, (double)x.y, a);
+  a = fma((double)wv.z, (double)x.z, a);
+  return fma((double)wv.w, (double)x.w, a);
+}
+
+// Whole router rows, one per chunk, of up to kRouterBatch consecutive chunks at once: each
+// thread takes float4 columns t + 512 j of every row, with an independent binary64 chain per
+// (row, j); one transposing warp reduction for all rows; the warp partials through shared
+// memory, summed in warp order by the batch's last warp, which stores the logits.
+constexpr int kRouterBatch = 4;
+
+__device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* sm, int u,
+                                             int r0, int nrows, const Ring& R, unsigned use0,
+                                             double* red, const XRouter& xr, bool last_of_cta) {
+  const int lane = threadIdx.x & 31;
+  const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
+  const int t = w * 32 + lane;
+  const int nf = G.rcols / 4;
+  double v[kRouterBatch];
+#pragma unroll
+  for (int r = 0; r < kRouterBatch; ++r) {
+    const float4* ws = reinterpret_cast<const float4*>(
+        ring_stage(G, R, use0 + (unsigned)(r < nrows ? r : 0)));
+    double p[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int f = t + kConsumers * j;
+      p[j] = (f < nf && r < nrows) ? row_dot4(ws, f, xr.v[j]) : 0.0;
+    }
+    v[r] = (p[0] + p[1]) + (p[2] + p[3]);
+  }
+  FMOE_MARK_W(u, MK_R_DOT, MK_R_DOT_W);
+  const int slot = ring_slot(R, use0);
+  double* rs = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(red) + (size_t)slot * G.red_slot);
+  seg_reduce<kRouterBatch>(v, lane, 32, [&](int r, double x) {
+    if (r < nrows) rs[r * kConsumerWarps + w] = x;
+  });
+  FMOE_MARK_W(u, MK_R_RED, MK_R_RED_W);
+  const bool last = chunk_last(sm, slot);
+  FMOE_MARK_W(u, MK_R_LAST, MK_R_LAST_W);
+  if (last) {
+    const double xf = (double)sm->xf[u & 1];
+    double* lg = P.s.logits + (size_t)(u & 1) * G.rseg * G.nr + r0;
+    if (lane < nrows) {
+      double x = 0.0;
+#pragma unroll
+      for (int q = 0; q < kConsumerWarps; ++q) x += rs[lane * kConsumerWarps + q];
+      lg[lane] = x * xf;  // the norm factor of x, applied to the sum
+    }
+    __syncwarp();
+    if (last_of_cta && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
+    FMOE_MARK(u, MK_R_PUB);
+  }
+  for (int r = 0; r < nrows; ++r) release_stage(ring_empty(R, use0 + (unsigned)r));
 }
 
 __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* sm,
@@ -1108,18 +1208,13 @@ __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* 
   const float4* ws = reinterpret_cast<const float4*>(stage);
   double* rs = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(red) + (size_t)slot * G.red_slot);
   for (int r = 0; r < c.n; ++r) {
-    double a = 0.0;
+    double p[4];
 #pragma unroll
-    for (int j = 0; j < 5; ++j) {
+    for (int j = 0; j < 4; ++j) {
       const int f = t + kConsumers * j;
-      if (f < nf) {
-        const float4 wv = ws[(size_t)r * nf + f];
-        a = fma((double)wv.x, xr.v[j][0], a);
-        a = fma((double)wv.y, xr.v[j][1], a);
-        a = fma((double)wv.z, xr.v[j][2], a);
-        a = fma((double)wv.w, xr.v[j][3], a);
-      }
+      p[j] = f < nf ? row_dot4(ws + (size_t)r * nf, f, xr.v[j]) : 0.0;
     }
+    double a = (p[0] + p[1]) + (p[2] + p[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
     if (lane == 0) rs[r * kConsumerWarps + w] = a;
@@ -1135,64 +1230,82 @@ __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* 
       lg[r] = a * xf;  // the norm factor of x, applied to the sum
     }
     __syncwarp();
-    if (last_of_cta && lane == 0 && !(P.debug & 1))
-      red_release_gpu(sig_word(P, SG_ROUTER), cta_rows);
+    if (last_of_cta && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
   }
   release_stage(empty);
   return true;
 }
 
-// Gate/up rows of a chunk: hr gate rows then hr up rows (n valid each) in the stage. Thread
-// (group g, slice s) takes rows rho = g + gh * i; partial sums are reduced over the row's
-// threads (lanes of its segment, then warps through shared memory); the chunk's last warp
-// applies SwiGLU and stores h. Returns whether the stage was handed back normally.
+// Gate/up rows of up to two chunks of one expert at once (a "pass"): chunk c's stage holds hr
+// gate rows then hr up rows (n_c valid each); row slot q = 2 hr c + rho. Thread (group g,
+// slice s) takes slots g + gh i (i < NR); every slot reads a copied row (row 0 of chunk 0
+// stands in for slots without a valid row), so the loads and products of all NR slots are
+// issued without branches. Partial sums are reduced over the row's threads (lanes of its
+// segment, then warps through shared memory); the pass's last warp applies SwiGLU, stores h
+// and, after the expert's last pass, publishes the CTA's progress on signal `sig`.
 template <int BITS, int FORM, int NR>
-__device__ __forceinline__ void gu_chunk(const Prog& P, const Geo& G, Smem* sm, const Chunk& c,
-                                         const uint8_t* stage, uint64_t* empty, int slot,
-                                         float* red, const typename XOf<FORM>::T& x, float* h,
-                                         int sig, bool last_of_k, unsigned cta_rows) {
+__device__ __forceinline__ void gu_pass(const Prog& P, const Geo& G, Smem* sm, int np,
+                                        const Chunk& c0, const Chunk& c1, const Ring& R,
+                                        unsigned use0, float* red,
+                                        const typename XOf<FORM>::T& x, float* h, int sig, int u,
+                                        bool last_of_k) {
+  const uint8_t* st0 = ring_stage(G, R, use0);
+  const uint8_t* st1 = ring_stage(G, R, use0 + (unsigned)(np - 1));
+  const int slot = ring_slot(R, use0);
   const int lane = threadIdx.x & 31;
   const int t = (int)threadIdx.x - 32 * kCtrlWarps;
   const int g = t / G.wh, s = t - g * G.wh;
   const bool act = g < G.gh && s < G.sh;
-  const int hr = G.hr, n = c.n;
+  const int sc = act ? s : 0;
+  const int hr = G.hr;
   constexpr unsigned cb = BITS == 4 ? 16u : 8u;
-  const uint32_t st = smem_u32(stage);
-  const uint32_t sb0 = st + 2u * (unsigned)hr * G.rc_h + (unsigned)(s >> 1) * 4u;
+  const unsigned sbo = 2u * (unsigned)hr * G.rc_h;  // offset of the sb words in a stage
   float acc[NR];
 #pragma unroll
   for (int i = 0; i < NR; ++i) {
-    acc[i] = 0.f;
-    const int rho = g + G.gh * i;
+    const int q = g + G.gh * i;
+    const int c = q >= 2 * hr ? 1 : 0;
+    const int rho = q - 2 * hr * c;
     const int rr = rho < hr ? rho : rho - hr;
-    if (act && rho < 2 * hr && rr < n) {
-      const uint32_t sbw = lds32(sb0 + (unsigned)rho * G.rs_h);
-      acc[i] = slice_any<BITS, FORM>(st + (unsigned)rho * G.rc_h + (unsigned)s * cb, sbw, x);
-    }
+    const bool ok = act && c < np && rr < (c ? c1.n : c0.n);
+    const int rc = ok ? rho : 0;
+    const uint8_t* st = (ok && c) ? st1 : st0;
+    const uint32_t sbw =
+        reinterpret_cast<const uint32_t*>(st + sbo)[(unsigned)rc * (G.rs_h >> 2) + (sc >> 1)];
+    const float v = slice_any<BITS, FORM>(st + (unsigned)rc * G.rc_h + (unsigned)sc * cb, sbw, x);
+    acc[i] = ok ? v : 0.f;
   }
-  // reduce over the row's threads: its segment of lanes, then (wide rows) its warps
+  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_DOT, MK_G_DOT_W);
+  // the stages are no longer read: reduce over the row's threads
   const int width = G.wh < 32 ? G.wh : 32;
   const int wn = G.wh > 32 ? G.wh / 32 : 1;  // warps per row group
   const int om = G.wh > 32 ? s >> 5 : 0;     // this warp's index within its group
   float* rs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + (size_t)slot * G.red_slot);
   seg_reduce<NR>(acc, lane & (width - 1), width, [&](int i, float v) {
-    const int rho = g + G.gh * i;
-    if (act && rho < 2 * hr) rs[rho * wn + om] = v;
+    const int q = g + G.gh * i;
+    if (act && q < 2 * hr * np) rs[q * wn + om] = v;
   });
+  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_RED, MK_G_RED_W);
   const bool last = chunk_last(sm, slot);
+  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_LAST, MK_G_LAST_W);
   if (last) {
-    for (int i = lane; i < n; i += 32) {
-      float a = 0.f, b = 0.f;
-      for (int q = 0; q < wn; ++q) {
-        a += rs[i * wn + q];
-        b += rs[(hr + i) * wn + q];
+    for (int c = 0; c < np; ++c) {
+      const int n = c ? c1.n : c0.n, r0 = c ? c1.r0 : c0.r0;
+      for (int i = lane; i < n; i += 32) {
+        float a = 0.f, b = 0.f;
+        for (int q = 0; q < wn; ++q) {
+          a += rs[(2 * hr * c + i) * wn + q];
+          b += rs[(2 * hr * c + hr + i) * wn + q];
+        }
+        h[r0 + i] = __fdividef(a, 1.f + __expf(-a)) * b;  // SwiGLU: SiLU(gate) * up
       }
-      h[c.r0 + i] = __fdividef(a, 1.f + __expf(-a)) * b;  // SwiGLU: SiLU(gate) * up
     }
     __syncwarp();
-    if (last_of_k && lane == 0) red_release_gpu(sig_word(P, sig), cta_rows);
+    if (last_of_k && lane == 0) publish(P, sig, u);
+    if (sig == SG_EXP0) FMOE_MARK(u, MK_G_PUB);
   }
-  release_stage(empty);
+  release_stage(ring_empty(R, use0));
+  if (np > 1) release_stage(ring_empty(R, use0 + 1));
 }
 
 // Down rows of a chunk (one expert segment): rows rho = w * P_i + lane_p + 8 P_i i of the
@@ -1208,26 +1321,29 @@ __device__ __forceinline__ void dn_chunk(const Geo& G, const Chunk& c, const uin
   const int lane_s = lane & (G.wi - 1), lane_p = lane / G.wi;
   const int n = c.n;
   constexpr unsigned cb = BITS == 4 ? 16u : 8u;
-  const uint32_t st = smem_u32(stage);
-  const uint32_t sbb = st + (unsigned)G.dr * G.rc_i;
+  const uint32_t* sbb = reinterpret_cast<const uint32_t*>(stage + (unsigned)G.dr * G.rc_i);
   float acc[NR];
 #pragma unroll
   for (int i = 0; i < NR; ++i) acc[i] = 0.f;
   for (int j = 0; j < G.ji; ++j) {
     const int s = lane_s + G.wi * j;
     const bool sok = s < G.si;
+    const int sc = sok ? s : 0;
     typename XOf<FORM>::T x;
     if constexpr (FORM == FORM_DIGITS)
-      load_digits(hseg, sok ? s : 0, x);
+      load_digits(hseg, sc, x);
     else
-      load_values(hseg, sok ? s : 0, hscale, x);
+      load_values(hseg, sc, hscale, x);
+    const uint8_t* code0 = stage + (unsigned)sc * cb;
+    const uint32_t* sbp = sbb + (sc >> 1);
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
       const int rho = w * G.pi + lane_p + kConsumerWarps * G.pi * i;
-      if (sok && rho < n) {
-        const uint32_t sbw = lds32(sbb + (unsigned)rho * G.rs_i + (unsigned)(s >> 1) * 4u);
-        acc[i] += slice_any<BITS, FORM>(st + (unsigned)rho * G.rc_i + (unsigned)s * cb, sbw, x);
-      }
+      const bool ok = sok && rho < n;
+      const int rc = ok ? rho : 0;  // row 0 stands in for slots without a valid row
+      const uint32_t sbw = sbp[(unsigned)rc * (G.rs_i >> 2)];
+      const float v = slice_any<BITS, FORM>(code0 + (unsigned)rc * G.rc_i, sbw, x);
+      acc[i] += ok ? v : 0.f;
     }
   }
   release_stage(empty);
@@ -1238,7 +1354,7 @@ __device__ __forceinline__ void dn_chunk(const Geo& G, const Chunk& c, const uin
   });
 }
 
-template <int BITS, int FORM, int NR>
+template <int BITS, int FORM, int NRG, int NRD>
 __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, const Share& S) {
   const int lane = threadIdx.x & 31;
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
@@ -1248,8 +1364,9 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
   float* red = reinterpret_cast<float*>(smem + G.o_red);
   float* oacc = reinterpret_cast<float*>(smem + G.o_oacc);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G.o_bar);
-  Ring A{smem + G.o_ringA, bars, bars + G.nA, G.nA, 0, 0u};
-  Ring B{smem + G.o_ringB, bars + 2 * G.nA, bars + 2 * G.nA + G.nB, G.nB, G.nA, 0u};
+  const Ring A{smem + G.o_ringA, bars, bars + G.nA, G.nA, 0};
+  const Ring B{smem + G.o_ringB, bars + 2 * G.nA, bars + 2 * G.nA + G.nB, G.nB, G.nA};
+  unsigned a_used = 0, b_used = 0;  // chunks taken from each ring so far
   const int gslice = t % G.wh;           // this thread's x slice in gate/up rows
   const bool gu_on = G.shared_on || G.routed_on;
   XRouter xr;
@@ -1262,117 +1379,136 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
   typename XOf<FORM>::T xg;              // x of this thread's slice (digits or values)
   for (int u = 0; u < P.n_units; ++u) {
     const int slot_u = u & 1;
+    const UnitView uv = unit_view(P, G, u);
+    const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
     if (!dead && !warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
       dead = true;
-    // ---- router rows
-    xr.seg = -1;
-    for (int i = 0; i < S.nrc; ++i) {
-      const Chunk c = chunk_a(G, S, i);
-      const unsigned st = A.used % (unsigned)A.ns;
-      if (!dead && !warp_wait_mbar(P, sm, &A.full[st], (A.used / (unsigned)A.ns) & 1u, DE_TIMEOUT_FULL))
+    if (w == 0) FMOE_MARK(u, MK_K_X);
+    // ---- router rows: whole rows in batches of up to kRouterBatch chunks, else chunk by chunk
+    if (G.route_on) {
+      if (S.nrc == 0) {
+        if (w == 0 && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
+      } else if (G.rseg == 1 && G.rrows == 1) {
+        const int bmax = min(kRouterBatch, A.ns);
+        for (int i0 = 0; i0 < S.nrc; i0 += bmax) {
+          const int nb = min(bmax, S.nrc - i0);
+          for (int q = 0; q < nb; ++q) ring_wait(P, sm, A, a_used + (unsigned)q, dead);
+          if (xr.seg != 0) router_x(G, XB, 0, xr);
+          router_batch(P, G, sm, u, S.r0 + i0, nb, A, a_used, reinterpret_cast<double*>(red), xr,
+                       i0 + nb == S.nrc);
+          a_used += (unsigned)nb;
+        }
+      } else {
+        xr.seg = -1;
+        for (int i = 0; i < S.nrc; ++i) {
+          const Chunk c = chunk_a(G, S, i);
+          ring_wait(P, sm, A, a_used, dead);
+          if (xr.seg != c.seg) router_x(G, XB, c.seg, xr);
+          router_chunk(P, G, sm, c, u, ring_stage(G, A, a_used), ring_empty(A, a_used),
+                       ring_slot(A, a_used), reinterpret_cast<double*>(red), xr, i == S.nrc - 1, 0u);
+          ++a_used;
+        }
+      }
+      xr.seg = -1;  // the next unit's x differs
+    }
+    if (w == 0) FMOE_MARK(u, MK_K_ROUTER);
+    // ---- x of this thread's slice: digit form (in place, after every router read of x)
+    if (gu_on) {
+      consumers_sync();
+      const float xf = sm->xf[slot_u];
+      if constexpr (FORM == FORM_DIGITS) {
+        transform<BITS>(XB, G.sh, xf);
+        consumers_sync();
+        load_digits(XB, gslice < G.sh ? gslice : 0, xg);
+      } else {
+        load_values(XB, gslice < G.sh ? gslice : 0, xf, xg);
+      }
+      // the x buffer is free once every warp holds its slice
+      if (lane == 0) {
+        const unsigned old = atom_add_acq_rel_cta_smem(&sm->xd_arrive, 1u);
+        if (old == (unsigned)(kConsumerWarps * (u + 1) - 1))
+          signal_ready(&sm->xfree, &sm->xfree_bar, (unsigned)(u + 1));
+      }
+      __syncwarp();
+      if (w == 0) FMOE_MARK(u, MK_K_XD);
+    }
+    // ---- routing decision: once every CTA's router rows of the unit are in
+    if (G.route_on) {
+      if (w == 0 && !dead &&
+          !warp_wait_sig(P, sm, SG_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE))
         dead = true;
-      if (xr.seg != c.seg) router_x(G, XB, c.seg, xr);
-      router_chunk(P, G, sm, c, u, A.base + (size_t)st * G.stage_bytes, &A.full[A.ns + st],
-                   A.slot0 + (int)st, reinterpret_cast<double*>(red), xr, i == S.nrc - 1,
-                   (unsigned)((S.r1 - S.r0) * G.rseg));
-      ++A.used;
+      consumers_sync();
+      if (w == 0) FMOE_MARK(u, MK_C_S1);
+      topk_block(P, G, sm, u, P.s.logits + (size_t)slot_u * G.rseg * G.nr, uv.bias,
+                 owner ? uv.idx_out : nullptr, owner ? uv.w_out : nullptr);
+      consumers_sync();
+      if (w == 0) FMOE_MARK(u, MK_C_RT);
     }
     if (!gu_on) continue;
-    // ---- x of this thread's slice: digit form (in place, after every router read of x)
-    consumers_sync();
-    const float xf = sm->xf[slot_u];
-    if constexpr (FORM == FORM_DIGITS) {
-      transform<BITS>(XB, G.sh, xf);
-      consumers_sync();
-      load_digits(XB, gslice < G.sh ? gslice : 0, xg);
-    } else {
-      load_values(XB, gslice < G.sh ? gslice : 0, xf, xg);
-    }
-    // the x buffer is free once every warp holds its slice
-    if (lane == 0) {
-      const unsigned old = atom_add_acq_rel_cta_smem(&sm->xd_arrive, 1u);
-      if (old == (unsigned)(kConsumerWarps * (u + 1) - 1))
-        signal_ready(&sm->xfree, &sm->xfree_bar, (unsigned)(u + 1));
-    }
-    __syncwarp();
-    const unsigned hrows = (unsigned)(S.h1 - S.h0);
-    // ---- shared expert: gate/up rows, then (once every CTA's are done) down rows
-    if (G.shared_on) {
-      for (int i = 0; i < S.ngc; ++i) {
-        const Chunk c = chunk_a(G, S, S.nrc + i);
-        const unsigned st = A.used % (unsigned)A.ns;
-        if (!dead && !warp_wait_mbar(P, sm, &A.full[st], (A.used / (unsigned)A.ns) & 1u, DE_TIMEOUT_FULL))
-          dead = true;
-        gu_chunk<BITS, FORM, NR>(P, G, sm, c, A.base + (size_t)st * G.stage_bytes,
-                                 &A.full[A.ns + st], A.slot0 + (int)st, red, xg,
-                                 P.s.hs + (size_t)slot_u * G.I, SG_SHARED, i == S.ngc - 1, hrows);
-        ++A.used;
+    // ---- gate/up rows: job 0 the shared expert (ring A), then routed expert k (ring B); each
+    // job in passes of up to gpass chunks
+    const int jobs = G.shared_on + (G.routed_on ? G.K : 0);
+    for (int job = 0; job < jobs; ++job) {
+      const bool sh = G.shared_on && job == 0;
+      const int k = job - G.shared_on;  // routed expert slot
+      const int sig = sh ? SG_SHARED : SG_EXP0 + k;
+      float* hdst = sh ? P.s.hs + (size_t)slot_u * G.I : P.s.hk + ((size_t)slot_u * G.K + k) * G.I;
+      const Ring R = sh ? A : B;
+      unsigned use = sh ? a_used : b_used;
+      if (S.ngc == 0 && w == 0 && lane == 0) publish(P, sig, u);
+      for (int i0 = 0; i0 < S.ngc; i0 += G.gpass) {
+        const int np = min(G.gpass, S.ngc - i0);
+        const Chunk c0 = sh ? chunk_a(G, S, S.nrc + i0) : chunk_b(G, S, k * S.ngc + i0);
+        const Chunk c1 = sh ? chunk_a(G, S, S.nrc + i0 + np - 1)
+                            : chunk_b(G, S, k * S.ngc + i0 + np - 1);
+        ring_wait(P, sm, R, use, dead);
+        if (np > 1) ring_wait(P, sm, R, use + 1, dead);
+        if (w == 0 && i0 == 0 && !sh) FMOE_MARK(u, MK_K_P2F + k);
+        gu_pass<BITS, FORM, NRG>(P, G, sm, np, c0, c1, R, use, red, xg, hdst, sig, u,
+                                 i0 + np == S.ngc);
+        use += (unsigned)np;
       }
-      if (S.ndc > 0) {
-        if (!dead && !warp_wait_ready(P, sm, &sm->hs_ready, &sm->hs_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
-          dead = true;
-        const float sg = sm->sigma[slot_u];
+      if (sh) a_used = use;
+      else b_used = use;
+      if (w == 0) FMOE_MARK(u, sh ? MK_K_SGU : MK_K_P2 + k);
+    }
+    // ---- down rows: segment 0 the shared expert (ring A), then routed expert k (ring B), each
+    // as soon as every CTA's h-rows of it are in; accumulated into this CTA's output rows
+    if (S.ndc > 0) {
+      for (int sgm = 0; sgm < G.nseg; ++sgm) {
+        const bool sh = G.shared_on && sgm == 0;
+        const int k = sgm - G.shared_on;
+        const bool okw = sh ? warp_wait_ready(P, sm, &sm->hs_ready, &sm->hs_bar, (unsigned)(u + 1),
+                                              DE_TIMEOUT_DEP)
+                            : warp_wait_ready(P, sm, &sm->hk_ready, &sm->hk_bar,
+                                              (unsigned)(u * G.K + k + 1), DE_TIMEOUT_DEP);
+        if (!dead && !okw) dead = true;
+        if (w == 0) FMOE_MARK(u, sh ? MK_K_HS : MK_K_HK + k);
+        float* hseg = HB + (size_t)sgm * G.I;
+        const float hsc = sh ? sm->sigma[slot_u] : sm->rt_w[slot_u][k];
         if constexpr (FORM == FORM_DIGITS) {
-          transform<BITS>(HB, G.si, sg);
+          transform<BITS>(hseg, G.si, hsc);
           consumers_sync();
         }
+        const Ring R = sh ? A : B;
+        unsigned use = sh ? a_used : b_used;
         for (int i = 0; i < S.ndc; ++i) {
-          const Chunk c = chunk_a(G, S, S.nrc + S.ngc + i);
-          const unsigned st = A.used % (unsigned)A.ns;
-          if (!dead && !warp_wait_mbar(P, sm, &A.full[st], (A.used / (unsigned)A.ns) & 1u,
-                                       DE_TIMEOUT_FULL))
-            dead = true;
-          dn_chunk<BITS, FORM, NR>(G, c, A.base + (size_t)st * G.stage_bytes, &A.full[A.ns + st],
-                                   HB, sg, oacc, S.d0);
-          ++A.used;
+          const Chunk c = sh ? chunk_a(G, S, S.nrc + S.ngc + i)
+                             : chunk_b(G, S, G.K * S.ngc + k * S.ndc + i);
+          ring_wait(P, sm, R, use, dead);
+          dn_chunk<BITS, FORM, NRD>(G, c, ring_stage(G, R, use), ring_empty(R, use), hseg, hsc,
+                                    oacc, S.d0);
+          ++use;
         }
-      }
-    }
-    // ---- routed experts: gate/up rows of k = 0..K-1, then down rows as each h_k completes
-    if (G.routed_on) {
-      for (int k = 0; k < G.K; ++k) {
-        float* hk = P.s.hk + ((size_t)slot_u * G.K + k) * G.I;
-        for (int i = 0; i < S.ngc; ++i) {
-          const Chunk c = chunk_b(G, S, k * S.ngc + i);
-          const unsigned st = B.used % (unsigned)B.ns;
-          if (!dead && !warp_wait_mbar(P, sm, &B.full[st], (B.used / (unsigned)B.ns) & 1u,
-                                       DE_TIMEOUT_FULL))
-            dead = true;
-          gu_chunk<BITS, FORM, NR>(P, G, sm, c, B.base + (size_t)st * G.stage_bytes,
-                                   &B.full[B.ns + st], B.slot0 + (int)st, red, xg, hk,
-                                   SG_EXP0 + k, i == S.ngc - 1, hrows);
-          ++B.used;
-        }
-      }
-      if (S.ndc > 0) {
-        for (int k = 0; k < G.K; ++k) {
-          if (!dead && !warp_wait_ready(P, sm, &sm->hk_ready, &sm->hk_bar,
-                                        (unsigned)(u * G.K + k + 1), DE_TIMEOUT_DEP))
-            dead = true;
-          float* hseg = HB + (size_t)(G.shared_on + k) * G.I;
-          const float wk = sm->rt_w[slot_u][k];
-          if constexpr (FORM == FORM_DIGITS) {
-            transform<BITS>(hseg, G.si, wk);
-            consumers_sync();
-          }
-          for (int i = 0; i < S.ndc; ++i) {
-            const Chunk c = chunk_b(G, S, G.K * S.ngc + k * S.ndc + i);
-            const unsigned st = B.used % (unsigned)B.ns;
-            if (!dead && !warp_wait_mbar(P, sm, &B.full[st], (B.used / (unsigned)B.ns) & 1u,
-                                         DE_TIMEOUT_FULL))
-              dead = true;
-            dn_chunk<BITS, FORM, NR>(G, c, B.base + (size_t)st * G.stage_bytes,
-                                     &B.full[B.ns + st], hseg, wk, oacc, S.d0);
-            ++B.used;
-          }
-        }
+        if (sh) a_used = use;
+        else b_used = use;
+        if (w == 0) FMOE_MARK(u, sh ? MK_K_DS : MK_K_D + k);
       }
     }
     // ---- outputs of this CTA's rows: residual + accumulated experts; sum of squares
-    if (G.nseg > 0 && S.d1 > S.d0) {
-      consumers_sync();
+    if (G.nseg > 0) {
+      if (S.d1 > S.d0) consumers_sync();
       if (w == 0) {
-        const UnitView uv = unit_view(P, G, u);
         float sq = 0.f;
         for (int r = S.d0 + lane; r < S.d1; r += 32) {
           const float o = (uv.res ? __ldcg(uv.res + r) : 0.f) + oacc[r - S.d0];
@@ -1380,13 +1516,14 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
           uv.out[r] = o;
           sq += o * o;
         }
-        if (P.mode == MODE_STACK) {
+        if (P.mode == MODE_STACK && S.d1 > S.d0) {
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
           if (lane == 0) atomicAdd(P.s.normsq + u, sq);
         }
         __syncwarp();
-        if (lane == 0) red_release_gpu(sig_word(P, SG_OUT), (unsigned)(S.d1 - S.d0));
+        if (lane == 0) publish(P, SG_OUT, u);
+        FMOE_MARK(u, MK_K_OUT);
       }
     }
   }
@@ -1432,12 +1569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     controller(P, G, smem, sm);
   } else {
-    const int nrg = (2 * G.hr + G.gh - 1) / G.gh;
-    const int nrd = (G.dr + kConsumerWarps * G.pi - 1) / (kConsumerWarps * G.pi);
-    if (max(nrg, nrd) <= 4)
-      consumer<BITS, FORM, 4>(P, G, smem, sm, S);
-    else
-      consumer<BITS, FORM, 8>(P, G, smem, sm, S);
+    consumer<BITS, FORM, kMaxRowsThread, kMaxRowsWarp>(P, G, smem, sm, S);
   }
 }
 

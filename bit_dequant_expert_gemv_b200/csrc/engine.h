@@ -18,8 +18,8 @@
 //   router (A) -> shared gate/up (A) -> shared down (A) -> routed gate/up k (B) -> routed down k (B)
 // with every warp taking part in every chunk. Cross-CTA dependencies are counted on monotone
 // global counters (one per signal, each on its own 128-byte line): a CTA adds the number of
-// rows it finished; signal s of unit u is complete when its counter reaches (u + 1) times the
-// rows of that phase.
+// rows it finished; signal s of unit u is complete when every CTA's word for s has reached
+// u + 1 (each CTA publishes its own progress word; no two CTAs write the same word).
 #pragma once
 #include <stdint.h>
 
@@ -32,12 +32,14 @@ constexpr int kThreads = kConsumers + 32 * kCtrlWarps;
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
 constexpr unsigned kStage = 18432;                 // bytes per ring stage
+constexpr int kRouterCols = 4 * 4 * 256;           // router columns per chunk (4 float4 per thread)
 constexpr int kMaxStages = 16;                     // per ring
 constexpr int kMaxRowsThread = 8;                  // gate/up rows one consumer thread holds
-constexpr int kMaxRowsWarp = 8;                    // down rows (per side-by-side lane group) a warp holds
+constexpr int kMaxRowsWarp = 4;                    // down rows (per side-by-side lane group) a warp holds
 constexpr int kMaxHr = 64;                         // h-rows per gate/up chunk (cap)
 
-// Global signals (counters in Scratch::ctrl, one 128-byte line each).
+// Global signals: per signal one progress word per CTA (Scratch::ctrl[s * kMaxCtas + cta]),
+// the number of units whose rows of that phase the CTA has finished.
 enum Sig {
   SG_ROUTER = 0,   // router rows finished (logits written)
   SG_SHARED = 1,   // shared-expert h-rows finished
@@ -45,7 +47,9 @@ enum Sig {
   SG_EXP0 = 3,     // + k: routed expert k's h-rows finished
   SG_COUNT = SG_EXP0 + kMaxK
 };
-constexpr int kCtrlWords = 32 * SG_COUNT;
+constexpr int kMaxCtas = 256;                      // grid size limit (one CTA per SM)
+constexpr int kCtrlWords = kMaxCtas * SG_COUNT;
+constexpr int kMiscBytes = 4096;                   // small shared state (Smem)
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
 
@@ -70,6 +74,7 @@ struct Geo {
   // gate/up chunks
   int au;                      // h-row alignment unit (rows whose sb bytes are a multiple of 16)
   int hr;                      // h-rows per chunk (a multiple of au)
+  int gpass;                   // gate/up chunks processed together (1 or 2)
   // down chunks
   int ad;                      // output-row alignment unit
   int dr;                      // output rows per chunk (a multiple of ad)
@@ -90,7 +95,7 @@ struct Geo {
 };
 
 struct Scratch {
-  unsigned* ctrl;        // kCtrlWords, zeroed per launch
+  unsigned* ctrl;        // kCtrlWords progress words, zeroed per launch
   int* err;              // sticky per-device error word
   double* logits;        // [2][rseg][nr] per unit parity: partial logits per column segment
   float* hs;             // [2][I]

@@ -241,7 +241,7 @@ int fmoe_stack_graph_destroy(fmoe_graph* graph);
     "H I E K bits route_on shared_on routed_on gate_on rc_h rs_h rc_i rs_i q_gu nr rseg rcols " \
     "rrows au hr ad dr nseg sh wh gh si wi pi ji stage_bytes nA nB o_ringA o_ringB o_x o_h "    \
     "o_red o_oacc o_misc o_bar oacc_n smem_bytes consumer_warps max_rows_thread max_rows_warp " \
-    "red_slot"
+    "red_slot gpass"
 int fmoe_describe_geometry(int hidden, int inter, int n_experts, int top_k, int bits, int flags,
                            int max_smem, int sms, int64_t* out, int n_out);
 

@@ -10,8 +10,7 @@ import pytest
 fmoe = pytest.importorskip("bit_dequant_expert_gemv_b200")
 
 MAX_SMEM = 232448
-WARPS = 8
-THREADS = 256
+MISC_BYTES = 4096
 
 SHAPES = [
     # H, I, E, K, bits
@@ -118,13 +117,17 @@ def inside(cov, a, nb):
     return any(lo <= a and a + nb <= hi for lo, hi in cov)
 
 
-def check_reads(G, kind, r0, n, seg, cov, NR, d0):
+def check_reads(G, kind, r0, n, seg, cov, d0):
+    """The consumer reads of one chunk; gate/up chunks are checked as chunk 0 or chunk 1 of a
+    pass (both positions), with the pass partner holding the same rows."""
+    WARPS = G["consumer_warps"]
+    THREADS = 32 * WARPS
     sb = G["stage_bytes"]
     cb = 16 if G["bits"] == 4 else 8
     if kind == CK_ROUTER:
         cols = G["rcols"]
         nf = cols // 4
-        assert nf <= 5 * THREADS  # the x columns a thread caches
+        assert nf <= 4 * THREADS  # the x columns a thread holds (4 float4)
         for r in range(n):
             for f in range(nf):
                 assert inside(cov, (r * nf + f) * 16, 16), (r, f)
@@ -132,25 +135,32 @@ def check_reads(G, kind, r0, n, seg, cov, NR, d0):
         assert (n * WARPS) * 8 <= G["red_slot"]
         return
     if kind == CK_GU:
+        NR = G["max_rows_thread"]
         hr, gh, wh, sh = G["hr"], G["gh"], G["wh"], G["sh"]
         wn = wh // 32 if wh > 32 else 1
         sb0 = 2 * hr * G["rc_h"]
-        for t in range(THREADS):
-            g, s = divmod(t, wh)
-            act = g < gh and s < sh
-            om = s >> 5 if wh > 32 else 0
-            for i in range(NR):
-                rho = g + gh * i
-                rr = rho if rho < hr else rho - hr
-                if act and rho < 2 * hr and rr < n:
-                    assert inside(cov, rho * G["rc_h"] + s * cb, cb), (t, rho, s)
-                    assert inside(cov, sb0 + rho * G["rs_h"] + (s >> 1) * 4, 4), (t, rho, s)
-                if act and rho < 2 * hr:
-                    assert (rho * wn + om) * 4 + 4 <= G["red_slot"]
-        # every valid row of the chunk is some thread's row
-        rows = {g + gh * i for g in range(gh) for i in range(NR)}
-        assert all(r in rows for r in range(n)) and all(hr + r in rows for r in range(n))
+        for np_, pos in [(1, 0)] + ([(2, 0), (2, 1)] if G["gpass"] == 2 else []):
+            seen = set()
+            for t in range(THREADS):
+                g, s = divmod(t, wh)
+                act = g < gh and s < sh
+                om = s >> 5 if wh > 32 else 0
+                for i in range(NR):
+                    q = g + gh * i
+                    c = 1 if q >= 2 * hr else 0
+                    rho = q - 2 * hr * c
+                    rr = rho if rho < hr else rho - hr
+                    if act and c < np_ and rr < n:
+                        if c == pos:  # a slot of this chunk reads its stage
+                            assert inside(cov, rho * G["rc_h"] + s * cb, cb), (t, rho, s)
+                            assert inside(cov, sb0 + rho * G["rs_h"] + (s >> 1) * 4, 4), (t, rho, s)
+                            seen.add(rho)
+                    if act and q < 2 * hr * np_:
+                        assert (q * wn + om) * 4 + 4 <= G["red_slot"]
+            # every valid row of the chunk is some thread's row
+            assert all(r in seen for r in range(n)) and all(hr + r in seen for r in range(n))
         return
+    NR = G["max_rows_warp"]
     wi, pi, ji, si = G["wi"], G["pi"], G["ji"], G["si"]
     sbb = G["dr"] * G["rc_i"]
     seen = set()
@@ -192,7 +202,7 @@ def check_geometry(G, nc):
     areas = [("ringA", G["o_ringA"], nA * sb), ("ringB", G["o_ringB"], nB * sb),
              ("x", G["o_x"], 4 * H), ("h", G["o_h"], max(4 * nseg * I, 128)),
              ("red", G["o_red"], G["red_slot"] * (nA + nB)), ("oacc", G["o_oacc"], 4 * max(G["oacc_n"], 1)),
-             ("misc", G["o_misc"], 512), ("bar", G["o_bar"], 16 * (nA + nB))]
+             ("misc", G["o_misc"], MISC_BYTES), ("bar", G["o_bar"], 16 * (nA + nB))]
     for (n1, a1, l1), (n2, a2, l2) in zip(areas, areas[1:]):
         assert a1 + l1 <= a2, (n1, n2)
     assert areas[-1][1] + areas[-1][2] <= G["smem_bytes"]
@@ -202,15 +212,15 @@ def check_geometry(G, nc):
     # the controller's bulk copies: x (4H bytes), each h segment (4I bytes at 4I k)
     assert (4 * H) % 16 == 0 and (4 * I) % 16 == 0
     # consumer layouts
+    THREADS = 32 * G["consumer_warps"]
     assert G["sh"] == H // 32 and G["gh"] * G["wh"] <= THREADS and G["gh"] >= 1
     assert G["wh"] >= G["sh"] and (G["wh"] <= 32 or G["wh"] % 32 == 0)
     if G["wh"] <= 32:
         assert G["wh"] & (G["wh"] - 1) == 0
     assert G["wi"] * G["pi"] == 32 and G["wi"] * G["ji"] >= G["si"]
-    nrg = -(-2 * G["hr"] // G["gh"])
-    nrd = -(-G["dr"] // (WARPS * G["pi"]))
-    assert max(nrg, nrd) <= 8
-    NR = 4 if max(nrg, nrd) <= 4 else 8
+    nrg = -(-2 * G["gpass"] * G["hr"] // G["gh"])
+    nrd = -(-G["dr"] // (G["consumer_warps"] * G["pi"]))
+    assert nrg <= G["max_rows_thread"] and nrd <= G["max_rows_warp"]
     # transform work items stay inside their vectors
     for bits_ts, nsl, length in [(4 if G["bits"] == 4 else 2, H // 32, H),
                                  (4 if G["bits"] == 4 else 2, I // 32, I)]:
@@ -245,7 +255,7 @@ def check_geometry(G, nc):
             key = (kind, n, seg, r0 - S["d0"] if kind == CK_DN else 0)
             if key not in checked:
                 checked.add(key)
-                check_reads(G, kind, r0, n, seg, cov, NR, S["d0"])
+                check_reads(G, kind, r0, n, seg, cov, S["d0"])
             if kind == CK_ROUTER:
                 covered_rows[CK_ROUTER] += [(r, seg) for r in range(r0, r0 + n)]
             else:
