@@ -218,7 +218,9 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
     return at;
   };
   const unsigned x_b = 4u * (unsigned)H;
-  const unsigned h_b = 4u * (unsigned)(G->nseg * I);
+  // the h area also holds the digit form of x (written by the controller while the router
+  // reads x, read by the consumers before any h value arrives)
+  const unsigned h_b = std::max(4u * (unsigned)(G->nseg * I), x_b);
   const unsigned wn = G->wh > 32 ? (unsigned)G->wh / 32 : 1u;
   const unsigned red_slot = std::max(8u * (unsigned)G->rrows * kConsumerWarps,
                                      4u * 2u * (unsigned)(G->gpass * G->hr) * wn);
@@ -272,32 +274,30 @@ int check_layer(const fmoe_layer_desc* L, const fmoe_layer_desc* L0) {
 
 // ---------------------------------------------------------------- scratch
 struct ScratchPlan {
-  size_t off_ctrl, off_normsq, zero_bytes, off_logits, off_hs, off_hk, off_hbuf, total;
+  size_t off_ctrl, off_logits, off_hx, off_hbuf, total;
 };
 
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
-ScratchPlan plan_scratch(const Geo& G, int n_units) {
+// Every part of the scratch is an exchange buffer that must start at zero (the whole plan is
+// zeroed before each launch); the stack buffer exists only for MODE_STACK programs.
+ScratchPlan plan_scratch(const Geo& G, int mode) {
   ScratchPlan s;
   size_t o = 0;
   s.off_ctrl = o; o = up256(o + 4 * (size_t)kCtrlWords);
-  s.off_normsq = o; o = up256(o + 4 * (size_t)n_units);
-  s.zero_bytes = o;
   s.off_logits = o; o = up256(o + 8 * 2 * (size_t)std::max(G.rseg, 1) * std::max(G.nr, 1));
-  s.off_hs = o; o = up256(o + 4 * 2 * (size_t)G.I);
-  s.off_hk = o; o = up256(o + 4 * 2 * (size_t)G.K * G.I);
-  s.off_hbuf = o; o = up256(o + 4 * 2 * (size_t)G.H);
+  s.off_hx = o; o = up256(o + 8 * 2 * (size_t)G.nseg * G.I);
+  s.off_hbuf = o; o = up256(o + (mode == MODE_STACK ? 8 * 2 * (size_t)G.H : 0));
   s.total = o;
   return s;
 }
 
 void bind_scratch(Prog* P, const ScratchPlan& sp, uint8_t* base, int* err) {
   P->s.ctrl = reinterpret_cast<unsigned*>(base + sp.off_ctrl);
-  P->s.normsq = reinterpret_cast<float*>(base + sp.off_normsq);
-  P->s.logits = reinterpret_cast<double*>(base + sp.off_logits);
-  P->s.hs = reinterpret_cast<float*>(base + sp.off_hs);
-  P->s.hk = reinterpret_cast<float*>(base + sp.off_hk);
-  P->s.hbuf = reinterpret_cast<float*>(base + sp.off_hbuf);
+  P->s.logits = reinterpret_cast<unsigned long long*>(base + sp.off_logits);
+  P->s.hx = reinterpret_cast<unsigned long long*>(base + sp.off_hx);
+  P->s.hbuf = sp.total > sp.off_hbuf ? reinterpret_cast<unsigned long long*>(base + sp.off_hbuf)
+                                     : nullptr;
   P->s.err = err;
 }
 
@@ -311,10 +311,10 @@ void fill_layers(Prog* P, const fmoe_layer_desc* layers, int n) {
   }
 }
 
-// Enqueue one engine run: zero the control words, launch.
+// Enqueue one engine run: zero the exchange buffers, launch.
 int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, int sms,
                    cudaStream_t st) {
-  CK(cudaMemsetAsync(base, 0, sp.zero_bytes, st));
+  CK(cudaMemsetAsync(base, 0, sp.total, st));
   cudaError_t e = fmoe_engine_launch(P, &G, sms, st);
   if (e != cudaSuccess) return cuda_fail(e, "engine launch");
   ++g_launches;
@@ -323,7 +323,7 @@ int enqueue_engine(Prog* P, const Geo& G, const ScratchPlan& sp, uint8_t* base, 
 
 // Run a program with scratch taken from the library's stream-ordered pool.
 int run_pooled(Prog* P, const Geo& G, DevState* d, cudaStream_t st) {
-  const ScratchPlan sp = plan_scratch(G, P->n_units);
+  const ScratchPlan sp = plan_scratch(G, P->mode);
   void* base = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&base, sp.total, d->pool, st);
   if (e != cudaSuccess) return fail(FMOE_ERR_NOMEM, "scratch allocation: %s", cudaGetErrorString(e));
@@ -630,7 +630,7 @@ int fmoe_moe_layer_noalloc(const fmoe_layer_desc* layer, const float* x, const f
   if (!aligned16(x) || !aligned16(out) || !aligned16(residual))
     return fail(FMOE_ERR_ALIGN, "x, residual, out must be 16-byte aligned");
   if (x == out) return fail(FMOE_ERR_INVALID, "x must not alias out");
-  const ScratchPlan sp = plan_scratch(G, 1);
+  const ScratchPlan sp = plan_scratch(G, MODE_SEQ);
   if (sp.total > kNoAllocErrOff)
     return fail(FMOE_ERR_UNSUPPORTED,
                 "fmoe_moe_layer_noalloc: this shape needs %zu bytes of scratch, the fixed area "
@@ -707,8 +707,7 @@ int fmoe_stack_graph_create(const fmoe_layer_desc* layers, int n_layers, const f
     return rc;
   if (tokens_per_launch <= 0 || tokens_per_launch > n_tokens) tokens_per_launch = n_tokens;
   const int H = G.H, E = G.E, K = G.K, L = n_layers;
-  const int units_per_launch = tokens_per_launch * L;
-  const ScratchPlan sp = plan_scratch(G, units_per_launch);
+  const ScratchPlan sp = plan_scratch(G, MODE_STACK);
   fmoe_graph* g = new fmoe_graph();
   cudaError_t e = cudaMalloc(&g->scratch, sp.total);
   if (e != cudaSuccess) {

@@ -58,7 +58,8 @@ enum MarkEv {
   MK_R_DOT = 67, MK_R_RED, MK_R_LAST, MK_R_PUB,   // router batch: first and last consumer warp
   MK_R_DOT_W = 71, MK_R_RED_W, MK_R_LAST_W,
   MK_G_DOT = 74, MK_G_RED, MK_G_LAST, MK_G_PUB,   // first gate/up pass of routed expert 0
-  MK_G_DOT_W = 78, MK_G_RED_W, MK_G_LAST_W
+  MK_G_DOT_W = 78, MK_G_RED_W, MK_G_LAST_W,
+  MK_J1_TOP = 81, MK_J1_W0, MK_B_I2, MK_B_I3, MK_G_EPI_END
 };
 // marks from the first (w == 0) and the last consumer warp inside a phase
 #define FMOE_MARK_W(u, ev0, evw)                                   \
@@ -73,7 +74,6 @@ enum MarkEv {
 // ------------------------------------------------------------------------------------------
 struct Smem {
   uint64_t xbar;               // the controller's bulk-copy barrier for x
-  uint64_t hbar;               // the controller's bulk-copy barrier for h
   // Readiness published by the controller (and one by the consumers): a monotone counter (the
   // truth) and an mbarrier that completes one phase per increment, used only to sleep until
   // the next increment.
@@ -83,6 +83,7 @@ struct Smem {
   unsigned hs_ready;           // units whose h_s is in the h buffer
   unsigned hk_ready;           // routed segments ready, counted over units: u*K + k + 1
   unsigned xfree;              // units whose x buffer the consumers no longer read
+  unsigned gu_issued;          // units whose routed gate/up copies producer B has all issued
   unsigned xd_arrive;          // consumer warps done loading x digits (8 per unit)
   unsigned chunk_arrive[2 * kMaxStages];  // per stage (ring A, then B): warps done with it
   float xf[2];                 // RMSNorm factor of the unit's x (1 without a norm)
@@ -101,29 +102,115 @@ __device__ __forceinline__ void raise_error(const Prog& P, Smem* sm, int code) {
   sm->abort = 1;
 }
 
-__device__ __forceinline__ unsigned* sig_row(const Prog& P, int s) {
-  return P.s.ctrl + (size_t)s * kMaxCtas;
+// ------------------------------------------------------------------------------------------
+// exchange words (see engine.h): tags, packing, unit-done words
+// ------------------------------------------------------------------------------------------
+constexpr unsigned long long kTag13 = 0x1FFFull;               // logit words: low mantissa bits
+constexpr unsigned long long kTag32 = 0xFFFFFFFF00000000ull;   // value words: high half
+
+__device__ __forceinline__ unsigned long long tag13(int u) {
+  return (unsigned long long)(u % 8191 + 1);
+}
+__device__ __forceinline__ unsigned long long tag32(int u) {
+  return (unsigned long long)(unsigned)(u + 1) << 32;
+}
+// A binary64 logit with the unit's tag in its 13 lowest mantissa bits (a change of at most
+// 2^-39 relative, inside the band where the top-K treats logits as tied).
+__device__ __forceinline__ unsigned long long logit_word(double l, int u) {
+  return ((unsigned long long)__double_as_longlong(l) & ~kTag13) | tag13(u);
+}
+__device__ __forceinline__ double logit_of(unsigned long long w) {
+  return __longlong_as_double((long long)(w & ~kTag13));
+}
+__device__ __forceinline__ unsigned long long value_word(float v, int u) {
+  return tag32(u) | (unsigned long long)__float_as_uint(v);
+}
+__device__ __forceinline__ float value_of(unsigned long long w) {
+  return __uint_as_float((unsigned)w);
 }
 
-// This CTA has finished its rows of signal s for units 0..u (one lane; after every write of
-// those rows by this CTA is ordered before it, e.g. by a CTA barrier or an acquire chain).
-__device__ __forceinline__ void publish(const Prog& P, int s, int u) {
-  st_release(sig_row(P, s) + blockIdx.x, (unsigned)(u + 1));
+// This lane: poll the word at p until its tag bits (mask) equal `want`, the budget runs out,
+// the CTA aborts or another CTA has recorded an error. Returns the last word read; if its tag
+// differs from `want`, the wait failed (and the failure is recorded).
+__device__ __noinline__ unsigned long long await_word(const Prog& P, Smem* sm,
+                                                      const unsigned long long* p,
+                                                      unsigned long long mask,
+                                                      unsigned long long want, int code) {
+  unsigned long long v = ld_relaxed_gpu_u64(p);
+  if ((v & mask) == want) return v;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+#pragma unroll 1
+  for (unsigned it = 0;; ++it) {
+    __nanosleep(32);
+    v = ld_relaxed_gpu_u64(p);
+    if ((v & mask) == want) return v;
+    if ((it & 7) == 7) {
+      if (sm->abort || ld_volatile_int(P.s.err) != 0) {
+        sm->abort = 1;
+        return v;
+      }
+      if (global_ns() > deadline) {
+        raise_error(P, sm, code);
+        return v;
+      }
+    }
+  }
+}
+
+// This lane's N words v[j] (already loaded from addr(j)): re-read every word whose tag bits
+// (mask) differ from `want`, all those loads in flight together, with a short sleep between
+// rounds, until every word matches, the budget runs out, the CTA aborts or another CTA has
+// recorded an error (the failure is then recorded). False on failure.
+template <int N, typename Addr>
+__device__ __forceinline__ bool settle(const Prog& P, Smem* sm, unsigned long long (&v)[N],
+                                       Addr addr, unsigned long long mask,
+                                       unsigned long long want, int code) {
+  unsigned miss = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) miss |= ((v[j] & mask) != want ? 1u : 0u) << j;
+  if (!miss) return true;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+#pragma unroll 1
+  for (unsigned it = 0;; ++it) {
+    __nanosleep(64);
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if ((miss >> j) & 1u) v[j] = ld_relaxed_gpu_u64(addr(j));
+    miss = 0;
+#pragma unroll
+    for (int j = 0; j < N; ++j) miss |= ((v[j] & mask) != want ? 1u : 0u) << j;
+    if (!miss) return true;
+    if ((it & 7) == 7) {
+      if (sm->abort || ld_volatile_int(P.s.err) != 0) {
+        sm->abort = 1;
+        return false;
+      }
+      if (global_ns() > deadline) {
+        raise_error(P, sm, code);
+        return false;
+      }
+    }
+  }
+}
+
+// This CTA has written every output row of units 0..u (one lane). Nothing is read through
+// this word: it only orders the start of the next unit after the end of this one.
+__device__ __forceinline__ void unit_done(const Prog& P, int u) {
+  st_relaxed_gpu(P.s.ctrl + blockIdx.x, (unsigned)(u + 1));
 }
 
 // ------------------------------------------------------------------------------------------
 // bounded waits
 // ------------------------------------------------------------------------------------------
-// Whole warp: spin until every CTA's progress word of signal s has reached `target` (wrap-
-// safe), the budget runs out, the CTA aborts or another CTA has recorded an error. Lane l
-// polls words 4l..4l+3 and 128+4l.. with relaxed 16-byte loads; once every word is there,
-// every lane makes one acquire fence.
-__device__ __noinline__ bool warp_wait_sig(const Prog& P, Smem* sm, int s, unsigned target,
-                                           int code) {
+// Whole warp: spin until every CTA's unit-done word has reached `target` (wrap-safe), the
+// budget runs out, the CTA aborts or another CTA has recorded an error. Lane l polls words
+// 4l..4l+3 and 128+4l.. with relaxed 16-byte loads.
+__device__ __noinline__ bool warp_wait_done(const Prog& P, Smem* sm, unsigned target, int code) {
   const int lane = threadIdx.x & 31;
   const int nc = gridDim.x;
-  const unsigned* row = sig_row(P, s);
+  const unsigned* row = P.s.ctrl;
   uint64_t deadline = 0;
+#pragma unroll 1
   for (unsigned it = 0;; ++it) {
     bool ok = true;
 #pragma unroll
@@ -137,10 +224,7 @@ __device__ __noinline__ bool warp_wait_sig(const Prog& P, Smem* sm, int s, unsig
         ok = ok && (w0 + 3 >= nc || (int)(v.w - target) >= 0);
       }
     }
-    if (__all_sync(0xffffffffu, ok)) {
-      fence_acq_rel_gpu();
-      return true;
-    }
+    if (__all_sync(0xffffffffu, ok)) return true;
     if (it == 0) deadline = global_ns() + P.wait_ns;
     int bad = 0;
     if (lane == 0 && (it & 7) == 7) {
@@ -175,6 +259,7 @@ __device__ __noinline__ bool wait_mbar(const Prog& P, Smem* sm, uint64_t* bar, u
                                        int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
+#pragma unroll 1
   for (unsigned it = 0;; ++it) {
     if (mbar_poll(bar, parity)) return true;
     if ((it & 7) == 7) {
@@ -194,6 +279,7 @@ __device__ __noinline__ bool wait_ready(const Prog& P, Smem* sm, const unsigned*
   unsigned c = ld_acquire_cta_smem(cnt);
   if ((int)(c - target) >= 0) return true;
   const uint64_t deadline = global_ns() + P.wait_ns;
+#pragma unroll 1
   for (unsigned it = 0;; ++it) {
     if (FMOE_WAIT_SUSPEND_NS > 0) {
       if (!mbar_try_wait_sleep(bar, c & 1u, FMOE_WAIT_SUSPEND_NS)) __nanosleep(64);
@@ -338,11 +424,14 @@ __device__ __forceinline__ Chunk chunk_b(const Geo& G, const Share& S, int i) {
 struct UnitView {
   int t, l, slot;
   const LayerW* L;
-  const float* xin;   // raw input h (x before the norm)
-  bool norm;          // x = rmsnorm(h) using normsq[u-1]
-  const float* res;   // nullable
-  float* out;
-  const float* bias;  // nullable [E]
+  const float* xin;                 // x from an input buffer (null: xw)
+  const unsigned long long* xw;     // x as the previous unit's tagged output words (stack
+                                    // layers after the first; x = rmsnorm of them)
+  const float* res;                 // residual from an input buffer (nullable)
+  const unsigned long long* resw;   // residual as tagged words (with xw)
+  float* out;                       // output to a result buffer (null: outw)
+  unsigned long long* outw;         // output as tagged words for the next layer
+  const float* bias;                // nullable [E]
   int* idx_out;
   float* w_out;
   float* h_trace;
@@ -351,11 +440,13 @@ struct UnitView {
 __device__ __forceinline__ UnitView unit_view(const Prog& P, const Geo& G, int u) {
   UnitView v;
   v.slot = u & 1;
+  v.xw = nullptr;
+  v.resw = nullptr;
+  v.outw = nullptr;
   if (P.mode == MODE_SEQ) {
     v.t = u;
     v.l = u % P.n_layers;
     v.xin = P.x + (size_t)u * G.H;
-    v.norm = false;
     v.res = P.res ? P.res + (size_t)u * G.H : nullptr;
     v.out = P.out + (size_t)u * G.H;
     v.bias = P.bias ? P.bias + (size_t)u * G.E : nullptr;
@@ -366,10 +457,21 @@ __device__ __forceinline__ UnitView unit_view(const Prog& P, const Geo& G, int u
     const int L = P.n_layers;
     v.t = u / L;
     v.l = u % L;
-    v.xin = v.l == 0 ? P.x + (size_t)v.t * G.H : P.s.hbuf + (size_t)((u - 1) & 1) * G.H;
-    v.norm = v.l > 0;
-    v.res = v.xin;
-    v.out = v.l == L - 1 ? P.out + (size_t)v.t * G.H : P.s.hbuf + (size_t)(u & 1) * G.H;
+    if (v.l == 0) {
+      v.xin = P.x + (size_t)v.t * G.H;
+      v.res = v.xin;
+    } else {
+      v.xin = nullptr;
+      v.res = nullptr;
+      v.xw = P.s.hbuf + (size_t)((u - 1) & 1) * G.H;
+      v.resw = v.xw;
+    }
+    if (v.l == L - 1) {
+      v.out = P.out + (size_t)v.t * G.H;
+    } else {
+      v.out = nullptr;
+      v.outw = P.s.hbuf + (size_t)(u & 1) * G.H;
+    }
     const size_t tl = (size_t)v.t * L + v.l;
     v.bias = P.bias ? P.bias + tl * G.E : nullptr;
     v.idx_out = P.idx_out ? P.idx_out + tl * G.K : nullptr;
@@ -444,35 +546,31 @@ __device__ __forceinline__ unsigned chunk_bytes(const Geo& G, const Chunk& c) {
   return (unsigned)c.n * (G.rc_i + G.rs_i);
 }
 
-// Issue one chunk into a stage: lane 0 waits for the stage to be free and registers the
-// bytes on its full barrier; lanes 0..3 issue the copies.
+// Issue one chunk into a stage (one thread): wait for the stage to be free, register the
+// chunk's bytes on its full barrier, issue its copies one after another. (Issuing from a
+// single thread whose warp has no other live lanes streams fastest: several lanes issuing one
+// copy each, or one lane of a full warp, measured markedly slower on this part.)
 __device__ __forceinline__ bool issue_chunk(const Prog& P, const Geo& G, Smem* sm,
                                             uint8_t* stage, uint64_t* full, uint64_t* empty,
                                             unsigned use, const LayerW& L, const uint8_t* eb,
                                             const Chunk& c) {
-  const int lane = threadIdx.x & 31;
-  int ok = 1;
-  if (lane == 0) {
-    ok = wait_mbar(P, sm, empty, (use & 1u) ^ 1u, DE_TIMEOUT_EMPTY);
-    if (ok) mbar_arrive_expect_tx(full, chunk_bytes(G, c));
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (!ok) return false;
-  if (lane < 4) {
+  if (!wait_mbar(P, sm, empty, (use & 1u) ^ 1u, DE_TIMEOUT_EMPTY)) return false;
+  mbar_arrive_expect_tx(full, chunk_bytes(G, c));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
     const uint8_t* src = nullptr;
     unsigned dst_off = 0;
-    const unsigned bytes = copy_desc(G, L, eb, c, lane, &src, &dst_off);
+    const unsigned bytes = copy_desc(G, L, eb, c, q, &src, &dst_off);
     if (bytes) tma_load_1d(stage + dst_off, src, bytes, full);
   }
-  __syncwarp();
   return true;
 }
 
 // Never leave the CTA with bulk copies in flight: wait for the last use of every stage.
 __device__ void drain_ring(const Prog& P, uint64_t* full, int ns, unsigned issued) {
-  if ((threadIdx.x & 31) != 0) return;
   const uint64_t deadline = global_ns() + 100000000ull;
   const unsigned first = issued > (unsigned)ns ? issued - (unsigned)ns : 0u;
+#pragma unroll 1
   for (unsigned j = first; j < issued; ++j) {
     while (!mbar_try_wait(&full[j % (unsigned)ns], (j / (unsigned)ns) & 1u)) {
       if (global_ns() > deadline) {
@@ -483,14 +581,63 @@ __device__ void drain_ring(const Prog& P, uint64_t* full, int ns, unsigned issue
   }
 }
 
+// Request chunks [i0, i1) of ring B's list for the unit routed to `rte` into L2 (one thread).
+__device__ __forceinline__ void prefetch_chunks_b(const Geo& G, const Share& S, const LayerW& L,
+                                                  const int* rte, int i0, int i1) {
+#pragma unroll 1
+  for (int i = i0; i < i1; ++i) {
+    const Chunk c = chunk_b(G, S, i);
+    const int e = min(max(rte[c.e], 0), G.E - 1);
+    const uint8_t* eb = L.experts + (size_t)e * L.expert_stride;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint8_t* src = nullptr;
+      unsigned dst_off = 0;
+      const unsigned bytes = copy_desc(G, L, eb, c, q, &src, &dst_off);
+      if (bytes) prefetch_l2_bulk(src, bytes);
+    }
+  }
+}
+
+// One thread: wait until the shared-memory counter *cnt reaches target (wrap-safe), bounded
+// like every other wait.
+__device__ __noinline__ bool wait_ready_counter(const Prog& P, Smem* sm, const unsigned* cnt,
+                                                unsigned target, int code) {
+  if ((int)(ld_acquire_cta_smem(cnt) - target) >= 0) return true;
+  const uint64_t deadline = global_ns() + P.wait_ns;
+#pragma unroll 1
+  for (unsigned it = 0;; ++it) {
+    __nanosleep(64);
+    if ((int)(ld_acquire_cta_smem(cnt) - target) >= 0) return true;
+    if ((it & 7) == 7) {
+      if (sm->abort) return false;
+      if (global_ns() > deadline) {
+        raise_error(P, sm, code);
+        return false;
+      }
+    }
+  }
+}
+
+// Producers run on one thread each (lane 0 of warps 0 and 1; the other lanes have left).
 __device__ void producer_a(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
                            const Share& S) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + G.o_bar);
   uint64_t* empty = full + G.nA;
   unsigned issued = 0;
   bool failed = false;
+  const bool gate = G.routed_on && S.nb > 0;
+#pragma unroll 1
   for (int u = 0; u < P.n_units && !failed; ++u) {
     const LayerW& L = P.layers[u % P.n_layers];
+    // The next unit's data-independent rows wait until the previous unit's routed gate/up
+    // copies are all out: they are needed later, and would otherwise share HBM with the
+    // stream that decides how soon the previous unit's gate/up rows are done.
+    if (gate && u > 0 && !wait_ready_counter(P, sm, &sm->gu_issued, (unsigned)u, DE_TIMEOUT_DEP)) {
+      failed = true;
+      break;
+    }
+#pragma unroll 1
     for (int i = 0; i < S.na; ++i) {
       const Chunk c = chunk_a(G, S, i);
       const unsigned st = issued % (unsigned)G.nA;
@@ -514,15 +661,27 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
   unsigned issued = 0;
   bool failed = false;
   if (S.nb == 0) return;
+#pragma unroll 1
   for (int u = 0; u < P.n_units && !failed; ++u) {
     const LayerW& L = P.layers[u % P.n_layers];
-    if (!warp_wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) {
+    if (!wait_ready(P, sm, &sm->rt_ready, &sm->rt_bar, (unsigned)(u + 1), DE_TIMEOUT_ROUTE)) {
       failed = true;
       break;
     }
     FMOE_MARK(u, MK_B_RT);
     const int* rte = sm->rt_e[u & 1];
+    // The first ring-full of chunks goes out first; then the gate/up copies that the ring
+    // cannot take yet are requested into L2 (so that HBM streams the CTA's whole routed
+    // gate/up share at once and the ring's later copies hit L2); the down copies follow the
+    // same way once every gate/up copy is out.
+    const int ngu = G.K * S.ngc;
+#pragma unroll 1
     for (int i = 0; i < S.nb; ++i) {
+      if (i == min(G.nB, ngu)) prefetch_chunks_b(G, S, L, rte, i, ngu);
+      if (i == ngu) {
+        st_release_cta_smem(&sm->gu_issued, (unsigned)(u + 1));
+        prefetch_chunks_b(G, S, L, rte, max(i, G.nB), S.nb);
+      }
       const Chunk c = chunk_b(G, S, i);
       const int e = min(max(rte[c.e], 0), G.E - 1);
       const uint8_t* eb = L.experts + (size_t)e * L.expert_stride;
@@ -533,8 +692,11 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
         break;
       }
       if (i == S.nb - 1) FMOE_MARK(u, MK_B_LAST);
+      if (i == 2) FMOE_MARK(u, MK_B_I2);
+      if (i == 3) FMOE_MARK(u, MK_B_I3);
       ++issued;
     }
+    if (ngu == S.nb) st_release_cta_smem(&sm->gu_issued, (unsigned)(u + 1));
   }
   if (failed) drain_ring(P, full, G.nB, issued);
 }
@@ -556,13 +718,16 @@ __device__ __forceinline__ unsigned long long pkey(double l, int e) {
   return (dkey(l) & ~0x1FFFull) | (unsigned long long)(0x1FFF - e);
 }
 
-// The binary64 logit of expert e: the bias first, then the column-segment partials in order.
-__device__ __forceinline__ double one_logit(const Geo& G, const double* lg, const float* bias,
-                                            int e) {
-  double l = ((double)(bias ? __ldcg(bias + e) : 0.f) + __ldcg(lg + e)) +
-             (G.rseg > 1 ? __ldcg(lg + (size_t)G.nr + e) : 0.0);
-  for (int sg = 2; sg < G.rseg; ++sg) l += __ldcg(lg + (size_t)sg * G.nr + e);
-  return l;
+// Word `sg` (column segment) of expert e's logit of unit u, polled until it carries the unit's
+// tag; `bad` is set if the wait failed.
+__device__ __forceinline__ double logit_part(const Prog& P, Smem* sm, const unsigned long long* lg,
+                                             unsigned long long wd, size_t at, int u, bool& bad) {
+  const unsigned long long want = tag13(u);
+  if ((wd & kTag13) != want) {
+    wd = await_word(P, sm, lg + at, kTag13, want, DE_TIMEOUT_ROUTE);
+    bad = bad || (wd & kTag13) != want;
+  }
+  return logit_of(wd);
 }
 
 // Top-K of the unit's logits by the consumer warps, after every CTA's router rows are in.
@@ -585,6 +750,7 @@ __device__ __forceinline__ void warp_topk(int K, unsigned long long (&key)[M], d
   const int lane = threadIdx.x & 31;
   out_key = 0ull;
   out_l = 0.0;
+#pragma unroll 1
   for (int k = 0; k < K; ++k) {
     unsigned long long bk = key[0];
     int bi = 0;
@@ -612,28 +778,65 @@ __device__ __forceinline__ void warp_topk(int K, unsigned long long (&key)[M], d
   }
 }
 
-__device__ __noinline__ void topk_block(const Prog& P, const Geo& G, Smem* sm, int u,
-                                        const double* lg, const float* bias, int* idx_out,
-                                        float* w_out) {
+__device__ __noinline__ bool topk_block(const Prog& P, const Geo& G, Smem* sm, int u,
+                                        const unsigned long long* lg, const float* bias,
+                                        int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
+  bool bad = false;
   float gate_l = 0.f;
   if (w == 0 && lane == 0 && G.gate_on) {  // the shared-gate row's logit (sigma), early
     double a = 0.0;
-    for (int sg = 0; sg < G.rseg; ++sg) a += __ldcg(lg + (size_t)sg * G.nr + G.E);
+#pragma unroll 1
+    for (int sg = 0; sg < G.rseg; ++sg) {
+      const size_t at = (size_t)sg * G.nr + G.E;
+      a += logit_part(P, sm, lg, ld_relaxed_gpu_u64(lg + at), at, u, bad);
+    }
     gate_l = (float)a;
   }
   unsigned long long best_key = 0ull;  // lane k < K: the warp's k-th best so far
   double best_l = 0.0;
   constexpr int kBlock = 64 * kConsumerWarps;
+#pragma unroll 1
   for (int e0 = 0; e0 < G.E; e0 += kBlock) {
     unsigned long long key[2];
     double lv[2];
+    int ec[2];
+    unsigned long long w0[2], w1[2];
+    float bv[2];
+    // words of the first two column segments of both experts: every load first, then one
+    // wait for all of them
+    const size_t s1 = G.rseg > 1 ? (size_t)G.nr : 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ec[i] = min(e0 + 32 * w + lane + 32 * kConsumerWarps * i, G.E - 1);
+      bv[i] = bias ? __ldcg(bias + ec[i]) : 0.f;
+    }
+    unsigned long long wd[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wd[j] = ld_relaxed_gpu_u64(lg + (j >> 1) * s1 + ec[j & 1]);
+    const int ec0 = ec[0], ec1 = ec[1];
+    if (!settle<4>(P, sm, wd, [=](int j) { return lg + (j >> 1) * s1 + ((j & 1) ? ec1 : ec0); }, kTag13,
+                   tag13(u), DE_TIMEOUT_ROUTE))
+      bad = true;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      w0[i] = wd[i];
+      w1[i] = wd[2 + i];
+    }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int e = e0 + 32 * w + lane + 32 * kConsumerWarps * i;
-      lv[i] = one_logit(G, lg, bias, min(e, G.E - 1));
-      key[i] = e < G.E ? pkey(lv[i], e) : 0ull;
+      // the bias first, then the column-segment partials in order
+      double l = (double)bv[i] + logit_of(w0[i]);
+      if (G.rseg > 1) l += logit_of(w1[i]);
+#pragma unroll 1
+      for (int sg = 2; sg < G.rseg; ++sg) {
+        const size_t at = (size_t)sg * G.nr + ec[i];
+        l += logit_part(P, sm, lg, ld_relaxed_gpu_u64(lg + at), at, u, bad);
+      }
+      lv[i] = l;
+      key[i] = e < G.E ? pkey(l, e) : 0ull;
     }
     unsigned long long bk;
     double bl;
@@ -649,12 +852,13 @@ __device__ __noinline__ void topk_block(const Prog& P, const Geo& G, Smem* sm, i
       warp_topk<2>(G.K, key, lv, best_key, best_l);
     }
   }
+  bad = __any_sync(0xffffffffu, bad);
   if (lane < G.K) {
     sm->cand_key[w * kMaxK + lane] = best_key;
     sm->cand_l[w * kMaxK + lane] = best_l;
   }
   consumers_sync();
-  if (w != 0) return;
+  if (w != 0) return bad;
   // merge: lane l holds candidates l + 32 i of the W K (missing ones are 0)
   constexpr int kM = (kConsumerWarps * kMaxK + 31) / 32;
   const int nc = kConsumerWarps * G.K;
@@ -685,112 +889,11 @@ __device__ __noinline__ void topk_block(const Prog& P, const Geo& G, Smem* sm, i
     if (idx_out) idx_out[lane] = e;
     if (w_out) w_out[lane] = wk;
   }
+  gate_l = __shfl_sync(0xffffffffu, gate_l, 0);
   if (lane == 0) sm->sigma[u & 1] = G.gate_on ? 1.f / (1.f + expf(-gate_l)) : 1.f;
   __syncwarp();
   if (lane == 0) signal_ready(&sm->rt_ready, &sm->rt_bar, (unsigned)(u + 1));
-}
-
-// ------------------------------------------------------------------------------------------
-// controller warp
-// ------------------------------------------------------------------------------------------
-// Bring `bytes` from global memory (written by other CTAs or by the caller) into shared
-// memory with one bulk copy issued by lane 0 on `bar`.
-__device__ __forceinline__ void copy_in(void* dst, const void* src, unsigned bytes,
-                                        uint64_t* bar) {
-  if ((threadIdx.x & 31) == 0) {
-    fence_proxy_async();  // order earlier generic accesses before the async-proxy copy
-    mbar_arrive_expect_tx(bar, bytes);
-    tma_load_1d(dst, src, bytes, bar);
-  }
-  __syncwarp();
-}
-
-__device__ __forceinline__ bool wait_copy(const Prog& P, Smem* sm, uint64_t* bar,
-                                          unsigned& phase) {
-  const bool ok = warp_wait_mbar(P, sm, bar, phase, DE_TIMEOUT_DEP);
-  phase ^= 1u;
-  return ok;
-}
-
-// The signal whose completion means "unit u is done" and its rows per unit.
-__device__ __forceinline__ int final_sig(const Geo& G) { return G.nseg > 0 ? SG_OUT : SG_ROUTER; }
-
-__device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm) {
-  const int lane = threadIdx.x & 31;
-  float* XB = reinterpret_cast<float*>(smem + G.o_x);
-  float* HB = reinterpret_cast<float*>(smem + G.o_h);
-  unsigned px = 0, ph = 0;  // phases of the x and h copy barriers
-  bool x_issued = false;    // the next unit's x copy is already in flight
-  const int fsig = final_sig(G);
-  const bool x_digits = G.shared_on || G.routed_on;
-  for (int u = 0; u < P.n_units; ++u) {
-    const UnitView uv = unit_view(P, G, u);
-    const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
-    FMOE_MARK(u, MK_C_UNIT);
-    // ---- x(u): computed on only after unit u-1 is complete everywhere
-    if (u > 0 && !warp_wait_sig(P, sm, fsig, (unsigned)u, DE_TIMEOUT_DEP)) break;
-    FMOE_MARK(u, MK_C_PREV_DONE);
-    if (!x_issued) copy_in(XB, uv.xin, 4u * (unsigned)G.H, &sm->xbar);
-    x_issued = false;
-    float f = 1.f;
-    if (uv.norm) f = rsqrtf(__ldcg(P.s.normsq + (u - 1)) / (float)G.H + P.eps);
-    if (!wait_copy(P, sm, &sm->xbar, px)) break;
-    FMOE_MARK(u, MK_C_X);
-    if (owner && uv.h_trace)
-      for (int c = lane * 4; c < G.H; c += 128)
-        *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XB + c);
-    if (lane == 0) {
-      sm->xf[u & 1] = f;
-      if (!G.route_on) sm->sigma[u & 1] = 1.f;
-      signal_ready(&sm->x_ready, &sm->x_bar, (unsigned)(u + 1));
-    }
-    __syncwarp();
-    if (G.route_on && uv.bias)  // the unit's logit bias into L2 while the router runs
-      for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
-    // ---- independent tokens: the next unit's x, once the consumers hold this unit's x
-    // digits in registers (its computation still waits for this unit to complete)
-    if (P.mode == MODE_SEQ && x_digits && u + 1 < P.n_units) {
-      if (!warp_wait_ready(P, sm, &sm->xfree, &sm->xfree_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
-        break;
-      FMOE_MARK(u, MK_C_XFREE);
-      copy_in(XB, P.x + (size_t)(u + 1) * G.H, 4u * (unsigned)G.H, &sm->xbar);
-      x_issued = true;
-    }
-    if (G.nseg == 0) continue;
-    // ---- h_s: every shared-expert h-row of unit u
-    if (G.shared_on) {
-      if (!warp_wait_sig(P, sm, SG_SHARED, (unsigned)(u + 1), DE_TIMEOUT_DEP)) break;
-      FMOE_MARK(u, MK_C_SS);
-      copy_in(HB, P.s.hs + (size_t)uv.slot * G.I, 4u * (unsigned)G.I, &sm->hbar);
-      if (!wait_copy(P, sm, &sm->hbar, ph)) break;
-      FMOE_MARK(u, MK_C_HS);
-      if (lane == 0) signal_ready(&sm->hs_ready, &sm->hs_bar, (unsigned)(u + 1));
-      __syncwarp();
-    }
-    // ---- h_k: routed expert k's h-rows of unit u, in order
-    if (G.routed_on) {
-      bool ok = true;
-      for (int k = 0; k < G.K && ok; ++k) {
-        ok = warp_wait_sig(P, sm, SG_EXP0 + k, (unsigned)(u + 1), DE_TIMEOUT_DEP);
-        if (!ok) break;
-        FMOE_MARK(u, MK_C_S2 + k);
-        copy_in(HB + (size_t)(G.shared_on + k) * G.I, P.s.hk + ((size_t)uv.slot * G.K + k) * G.I,
-                4u * (unsigned)G.I, &sm->hbar);
-        ok = wait_copy(P, sm, &sm->hbar, ph);
-        if (!ok) break;
-        FMOE_MARK(u, MK_C_HK + k);
-        if (lane == 0) signal_ready(&sm->hk_ready, &sm->hk_bar, (unsigned)(u * G.K + k + 1));
-        __syncwarp();
-      }
-      if (!ok) break;
-    }
-  }
-  // never leave with a copy in flight
-  if (x_issued && lane == 0) {
-    const uint64_t deadline = global_ns() + 100000000ull;
-    while (!mbar_try_wait(&sm->xbar, px))
-      if (global_ns() > deadline) break;
-  }
+  return bad;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -835,25 +938,26 @@ __device__ __forceinline__ int word_col(int n, int b) {
   return BITS == 4 ? 8 * (n >> 1) + 2 * b + (n & 1) : 16 * (n >> 2) + 4 * b + (n & 3);
 }
 
-// Transform nsl slices of buf (binary32, scaled by `scale`) into digit form, in place, by the
-// 256 consumer threads: 8 threads per slice, thread n of a slice making digit word n of the
-// three planes from its four columns. The 8 threads of a slice are consecutive lanes of one
-// warp, and every lane reads its values before any lane writes.
+// Transform nsl slices of src (binary32, scaled by `scale`) into digit form in dst (dst may
+// be src: in place), by nthr threads (tid = this thread's index among them, nthr a multiple of
+// 32, the threads whole warps): 8 threads per slice, thread n of a slice making digit word n
+// of the three planes from its four columns. The 8 threads of a slice are consecutive lanes of
+// one warp, and every lane reads its values before any lane writes.
 template <int BITS>
-__device__ void transform(float* buf, int nsl, float scale) {
-  const int t = (int)threadIdx.x - 32 * kCtrlWarps;
+__device__ void transform(const float* src, float* dst, int nsl, float scale, int tid, int nthr) {
   const int items = nsl * 8;
-  const int rounds = (items + kConsumers - 1) / kConsumers;
-  uint32_t* base = reinterpret_cast<uint32_t*>(buf);
+  const int rounds = (items + nthr - 1) / nthr;
+  uint32_t* base = reinterpret_cast<uint32_t*>(dst);
+#pragma unroll 1
   for (int r = 0; r < rounds; ++r) {
-    const int it = t + kConsumers * r;
+    const int it = tid + nthr * r;
     const bool act = it < items;
     const int s = act ? it >> 3 : 0, n = it & 7;
     float v[4];
     float m = 0.f, sum = 0.f;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      v[b] = act ? buf[32 * s + word_col<BITS>(n, b)] * scale : 0.f;
+      v[b] = act ? src[32 * s + word_col<BITS>(n, b)] * scale : 0.f;
       m = fmaxf(m, fabsf(v[b]));
     }
     sum = (v[0] + v[1]) + (v[2] + v[3]);
@@ -880,6 +984,12 @@ __device__ void transform(float* buf, int nsl, float scale) {
     }
     __syncwarp();
   }
+}
+
+// The consumers' form: all 256 consumer threads, in place.
+template <int BITS>
+__device__ __forceinline__ void transform(float* buf, int nsl, float scale) {
+  transform<BITS>(buf, buf, nsl, scale, (int)threadIdx.x - 32 * kCtrlWarps, kConsumers);
 }
 
 // The digit form of slice s of buf: xd[8p + n] = word n of plane p; {sc, sx}.
@@ -911,6 +1021,121 @@ __device__ __forceinline__ void load_values(const float* buf, int s, float scale
     const float4 a = *reinterpret_cast<const float4*>(buf + 32 * s + 4 * q);
     x.v[4 * q] = a.x * scale; x.v[4 * q + 1] = a.y * scale;
     x.v[4 * q + 2] = a.z * scale; x.v[4 * q + 3] = a.w * scale;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// controller warp
+// ------------------------------------------------------------------------------------------
+// Bring `bytes` from global memory (written by other CTAs or by the caller) into shared
+// memory with one bulk copy issued by lane 0 on `bar`.
+__device__ __forceinline__ void copy_in(void* dst, const void* src, unsigned bytes,
+                                        uint64_t* bar) {
+  if ((threadIdx.x & 31) == 0) {
+    fence_proxy_async();  // order earlier generic accesses before the async-proxy copy
+    mbar_arrive_expect_tx(bar, bytes);
+    tma_load_1d(dst, src, bytes, bar);
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ bool wait_copy(const Prog& P, Smem* sm, uint64_t* bar,
+                                          unsigned& phase) {
+  const bool ok = warp_wait_mbar(P, sm, bar, phase, DE_TIMEOUT_DEP);
+  phase ^= 1u;
+  return ok;
+}
+
+// Whole warp: the n tagged value words of unit u at src into dst as binary32, 16 words per
+// lane in flight; each word polled until it carries the unit's tag. False if a wait failed.
+__device__ __noinline__ bool fetch_values(const Prog& P, Smem* sm, const unsigned long long* src,
+                                          float* dst, int n, int u, int code) {
+  const int lane = threadIdx.x & 31;
+  const unsigned long long want = tag32(u);
+  bool ok = true;
+#pragma unroll 1
+  for (int b = 0; b < n; b += 32 * 16) {
+    const unsigned long long* sb = src + b + lane;
+    const int lim = n - 1 - b - lane;  // words j with 32 j <= lim are inside the vector
+    unsigned long long v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = ld_relaxed_gpu_u64(sb + min(32 * j, lim));
+    ok = settle<16>(P, sm, v, [=](int j) { return sb + min(32 * j, lim); }, kTag32, want, code) &&
+         ok;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (32 * j <= lim) dst[b + lane + 32 * j] = value_of(v[j]);
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, bool need_h) {
+  const int lane = threadIdx.x & 31;
+  float* XB = reinterpret_cast<float*>(smem + G.o_x);
+  float* HB = reinterpret_cast<float*>(smem + G.o_h);
+  unsigned px = 0;          // phase of the x copy barrier
+  bool x_issued = false;    // the next unit's x copy is already in flight
+  const bool x_digits = G.shared_on || G.routed_on;
+#pragma unroll 1
+  for (int u = 0; u < P.n_units; ++u) {
+    const UnitView uv = unit_view(P, G, u);
+    const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
+    FMOE_MARK(u, MK_C_UNIT);
+    // ---- x(u) from an input buffer: computed on only after unit u-1 is done everywhere
+    // (stack layers after the first read the previous layer's words in the consumers)
+    if (uv.xin) {
+      if (u > 0 && !warp_wait_done(P, sm, (unsigned)u, DE_TIMEOUT_DEP)) break;
+      FMOE_MARK(u, MK_C_PREV_DONE);
+      if (!x_issued) copy_in(XB, uv.xin, 4u * (unsigned)G.H, &sm->xbar);
+      x_issued = false;
+      if (!wait_copy(P, sm, &sm->xbar, px)) break;
+      FMOE_MARK(u, MK_C_X);
+      if (owner && uv.h_trace)
+#pragma unroll 1
+        for (int c = lane * 4; c < G.H; c += 128)
+          *reinterpret_cast<float4*>(uv.h_trace + c) = *reinterpret_cast<const float4*>(XB + c);
+      if (lane == 0) {
+        sm->xf[u & 1] = 1.f;
+        signal_ready(&sm->x_ready, &sm->x_bar, (unsigned)(u + 1));
+      }
+      __syncwarp();
+    }
+    if (G.route_on && uv.bias)  // the unit's logit bias into L2 while the router runs
+#pragma unroll 1
+      for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
+    // ---- independent tokens: the next unit's x, once the consumers hold this unit's x
+    // digits in registers (its computation still waits for this unit to complete)
+    if (P.mode == MODE_SEQ && x_digits && u + 1 < P.n_units) {
+      if (!warp_wait_ready(P, sm, &sm->xfree, &sm->xfree_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
+        break;
+      FMOE_MARK(u, MK_C_XFREE);
+      copy_in(XB, P.x + (size_t)(u + 1) * G.H, 4u * (unsigned)G.H, &sm->xbar);
+      x_issued = true;
+    }
+    if (G.nseg == 0 || !need_h) continue;  // (no output rows: no h needed)
+    // ---- h of unit u, segment by segment (shared expert, then routed k), as its words arrive
+    bool ok = true;
+#pragma unroll 1
+    for (int sg = 0; sg < G.nseg && ok; ++sg) {
+      const bool sh = G.shared_on && sg == 0;
+      const int k = sg - G.shared_on;
+      ok = fetch_values(P, sm, P.s.hx + ((size_t)uv.slot * G.nseg + sg) * G.I,
+                        HB + (size_t)sg * G.I, G.I, u, DE_TIMEOUT_DEP);
+      if (!ok) break;
+      FMOE_MARK(u, sh ? MK_C_HS : MK_C_HK + k);
+      if (lane == 0) {
+        if (sh) signal_ready(&sm->hs_ready, &sm->hs_bar, (unsigned)(u + 1));
+        else signal_ready(&sm->hk_ready, &sm->hk_bar, (unsigned)(u * G.K + k + 1));
+      }
+      __syncwarp();
+    }
+    if (!ok) break;
+  }
+  // never leave with a copy in flight
+  if (x_issued && lane == 0) {
+    const uint64_t deadline = global_ns() + 100000000ull;
+    while (!mbar_try_wait(&sm->xbar, px))
+      if (global_ns() > deadline) break;
   }
 }
 
@@ -1056,6 +1281,7 @@ __device__ __forceinline__ void seg_reduce(T (&v)[NR], int lane_in_seg, int widt
     }
   }
   if (nlive == 1) {
+#pragma unroll 1
     for (int o = NR; o < width; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
     if (lane_in_seg < NR && lane_in_seg < width) store(lo, v[0]);
   } else {
@@ -1117,32 +1343,24 @@ __device__ __forceinline__ void release_stage(uint64_t* empty) {
 // Router rows of a chunk: binary64 sums of fp32 products over the chunk's columns; each
 // thread takes float4 columns t, t + 256, ...; per row a warp reduction, the 8 warp
 // partials through shared memory, summed in warp order by the chunk's last warp.
-// This thread's x columns (float4 t + 512 j, j < 4) of the router segment it last loaded.
-struct XRouter {
-  float4 v[4];
-  int seg;          // which segment they hold (-1: none)
+// The x columns (float4 group f) of router segment `seg`, converted to binary64.
+struct X4 {
+  double a, b, c, d;
 };
 
-__device__ __forceinline__ void router_x(const Geo& G, const float* XB, int seg, XRouter& xr) {
-  const int t = (int)threadIdx.x - 32 * kCtrlWarps;
-  const int nf = G.rcols / 4;
-  const float4* xs = reinterpret_cast<const float4*>(XB + (size_t)seg * G.rcols);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int f = t + kConsumers * j;
-    xr.v[j] = f < nf ? xs[f] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  xr.seg = seg;
+__device__ __forceinline__ X4 router_x4(const Geo& G, const float* XB, int seg, int f) {
+  const float4 v = reinterpret_cast<const float4*>(XB + (size_t)seg * G.rcols)[f];
+  return X4{(double)v.x, (double)v.y, (double)v.z, (double)v.w};
 }
 
-// sum over the float4 columns of one row: four products each, converted to binary64 (exact)
-// and accumulated in binary64
-__device__ __forceinline__ double row_dot4(const float4* ws, int f, const float4& x) {
+// four products of one row's float4 group f with x, the weights converted to binary64 (the
+// products are exact), accumulated in binary64 onto `acc`
+__device__ __forceinline__ double row_dot4(const float4* ws, int f, const X4& x, double acc) {
   const float4 wv = ws[f];
-  double a = (double)wv.x * (double)x.x;
-  a = fma((double)wv.y, (double)x.y, a);
-  a = fma((double)wv.z, (double)x.z, a);
-  return fma((double)wv.w, (double)x.w, a);
+  acc = fma((double)wv.x, x.a, acc);
+  acc = fma((double)wv.y, x.b, acc);
+  acc = fma((double)wv.z, x.c, acc);
+  return fma((double)wv.w, x.d, acc);
 }
 
 // Whole router rows, one per chunk, of up to kRouterBatch consecutive chunks at once: each
@@ -1153,23 +1371,26 @@ constexpr int kRouterBatch = 4;
 
 __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* sm, int u,
                                              int r0, int nrows, const Ring& R, unsigned use0,
-                                             double* red, const XRouter& xr, bool last_of_cta) {
+                                             double* red, const float* XB) {
   const int lane = threadIdx.x & 31;
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
   const int t = w * 32 + lane;
   const int nf = G.rcols / 4;
   double v[kRouterBatch];
 #pragma unroll
-  for (int r = 0; r < kRouterBatch; ++r) {
-    const float4* ws = reinterpret_cast<const float4*>(
-        ring_stage(G, R, use0 + (unsigned)(r < nrows ? r : 0)));
-    double p[4];
+  for (int r = 0; r < kRouterBatch; ++r) v[r] = 0.0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int f = t + kConsumers * j;
-      p[j] = (f < nf && r < nrows) ? row_dot4(ws, f, xr.v[j]) : 0.0;
+  for (int j = 0; j < 4; ++j) {
+    const int f = t + kConsumers * j;
+    if (f < nf) {
+      const X4 x = router_x4(G, XB, 0, f);
+#pragma unroll
+      for (int r = 0; r < kRouterBatch; ++r) {
+        const float4* ws = reinterpret_cast<const float4*>(
+            ring_stage(G, R, use0 + (unsigned)(r < nrows ? r : 0)));
+        if (r < nrows) v[r] = row_dot4(ws, f, x, v[r]);
+      }
     }
-    v[r] = (p[0] + p[1]) + (p[2] + p[3]);
   }
   FMOE_MARK_W(u, MK_R_DOT, MK_R_DOT_W);
   const int slot = ring_slot(R, use0);
@@ -1182,39 +1403,37 @@ __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* 
   FMOE_MARK_W(u, MK_R_LAST, MK_R_LAST_W);
   if (last) {
     const double xf = (double)sm->xf[u & 1];
-    double* lg = P.s.logits + (size_t)(u & 1) * G.rseg * G.nr + r0;
-    if (lane < nrows) {
+    unsigned long long* lg = P.s.logits + (size_t)(u & 1) * G.rseg * G.nr + r0;
+    if (lane < nrows && !(P.debug & 1)) {  // debug bit 0: the logits are never written
       double x = 0.0;
 #pragma unroll
       for (int q = 0; q < kConsumerWarps; ++q) x += rs[lane * kConsumerWarps + q];
-      lg[lane] = x * xf;  // the norm factor of x, applied to the sum
+      st_relaxed_gpu_u64(lg + lane, logit_word(x * xf, u));  // norm factor applied to the sum
     }
-    __syncwarp();
-    if (last_of_cta && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
     FMOE_MARK(u, MK_R_PUB);
   }
+#pragma unroll 1
   for (int r = 0; r < nrows; ++r) release_stage(ring_empty(R, use0 + (unsigned)r));
 }
 
 __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* sm,
                                              const Chunk& c, int u, const uint8_t* stage,
                                              uint64_t* empty, int slot, double* red,
-                                             const XRouter& xr, bool last_of_cta,
-                                             unsigned cta_rows) {
+                                             const float* XB) {
   const int lane = threadIdx.x & 31;
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
   const int t = w * 32 + lane;
   const int nf = G.rcols / 4;
   const float4* ws = reinterpret_cast<const float4*>(stage);
   double* rs = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(red) + (size_t)slot * G.red_slot);
+#pragma unroll 1
   for (int r = 0; r < c.n; ++r) {
-    double p[4];
+    double a = 0.0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int f = t + kConsumers * j;
-      p[j] = f < nf ? row_dot4(ws + (size_t)r * nf, f, xr.v[j]) : 0.0;
+      if (f < nf) a = row_dot4(ws + (size_t)r * nf, f, router_x4(G, XB, c.seg, f), a);
     }
-    double a = (p[0] + p[1]) + (p[2] + p[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
     if (lane == 0) rs[r * kConsumerWarps + w] = a;
@@ -1222,15 +1441,14 @@ __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* 
   const bool last = chunk_last(sm, slot);
   if (last) {
     const double xf = (double)sm->xf[u & 1];
-    double* lg = P.s.logits + ((size_t)(u & 1) * G.rseg + c.seg) * G.nr + c.r0;
-    for (int r = lane; r < c.n; r += 32) {
+    unsigned long long* lg = P.s.logits + ((size_t)(u & 1) * G.rseg + c.seg) * G.nr + c.r0;
+#pragma unroll 1
+    for (int r = lane; r < c.n && !(P.debug & 1); r += 32) {
       double a = 0.0;
 #pragma unroll
       for (int q = 0; q < kConsumerWarps; ++q) a += rs[r * kConsumerWarps + q];
-      lg[r] = a * xf;  // the norm factor of x, applied to the sum
+      st_relaxed_gpu_u64(lg + r, logit_word(a * xf, u));  // norm factor applied to the sum
     }
-    __syncwarp();
-    if (last_of_cta && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
   }
   release_stage(empty);
   return true;
@@ -1241,14 +1459,14 @@ __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* 
 // slice s) takes slots g + gh i (i < NR); every slot reads a copied row (row 0 of chunk 0
 // stands in for slots without a valid row), so the loads and products of all NR slots are
 // issued without branches. Partial sums are reduced over the row's threads (lanes of its
-// segment, then warps through shared memory); the pass's last warp applies SwiGLU, stores h
-// and, after the expert's last pass, publishes the CTA's progress on signal `sig`.
+// segment, then warps through shared memory); the pass's last warp applies SwiGLU and stores
+// the h values as tagged words of unit u. `tr` marks the pass traced by a profiling build.
 template <int BITS, int FORM, int NR>
 __device__ __forceinline__ void gu_pass(const Prog& P, const Geo& G, Smem* sm, int np,
                                         const Chunk& c0, const Chunk& c1, const Ring& R,
                                         unsigned use0, float* red,
-                                        const typename XOf<FORM>::T& x, float* h, int sig, int u,
-                                        bool last_of_k) {
+                                        const typename XOf<FORM>::T& x, unsigned long long* h,
+                                        int u, bool tr) {
   const uint8_t* st0 = ring_stage(G, R, use0);
   const uint8_t* st1 = ring_stage(G, R, use0 + (unsigned)(np - 1));
   const int slot = ring_slot(R, use0);
@@ -1275,7 +1493,7 @@ __device__ __forceinline__ void gu_pass(const Prog& P, const Geo& G, Smem* sm, i
     const float v = slice_any<BITS, FORM>(st + (unsigned)rc * G.rc_h + (unsigned)sc * cb, sbw, x);
     acc[i] = ok ? v : 0.f;
   }
-  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_DOT, MK_G_DOT_W);
+  if (tr) FMOE_MARK_W(u, MK_G_DOT, MK_G_DOT_W);
   // the stages are no longer read: reduce over the row's threads
   const int width = G.wh < 32 ? G.wh : 32;
   const int wn = G.wh > 32 ? G.wh / 32 : 1;  // warps per row group
@@ -1285,25 +1503,28 @@ __device__ __forceinline__ void gu_pass(const Prog& P, const Geo& G, Smem* sm, i
     const int q = g + G.gh * i;
     if (act && q < 2 * hr * np) rs[q * wn + om] = v;
   });
-  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_RED, MK_G_RED_W);
+  if (tr) FMOE_MARK_W(u, MK_G_RED, MK_G_RED_W);
   const bool last = chunk_last(sm, slot);
-  if (sig == SG_EXP0) FMOE_MARK_W(u, MK_G_LAST, MK_G_LAST_W);
+  if (tr) FMOE_MARK_W(u, MK_G_LAST, MK_G_LAST_W);
   if (last) {
+#pragma unroll 1
     for (int c = 0; c < np; ++c) {
       const int n = c ? c1.n : c0.n, r0 = c ? c1.r0 : c0.r0;
+#pragma unroll 1
       for (int i = lane; i < n; i += 32) {
         float a = 0.f, b = 0.f;
+#pragma unroll 1
         for (int q = 0; q < wn; ++q) {
           a += rs[(2 * hr * c + i) * wn + q];
           b += rs[(2 * hr * c + hr + i) * wn + q];
         }
-        h[r0 + i] = __fdividef(a, 1.f + __expf(-a)) * b;  // SwiGLU: SiLU(gate) * up
+        // SwiGLU: SiLU(gate) * up
+        st_relaxed_gpu_u64(h + r0 + i, value_word(__fdividef(a, 1.f + __expf(-a)) * b, u));
       }
     }
-    __syncwarp();
-    if (last_of_k && lane == 0) publish(P, sig, u);
-    if (sig == SG_EXP0) FMOE_MARK(u, MK_G_PUB);
+    if (tr) FMOE_MARK(u, MK_G_PUB);
   }
+  if (tr && last) FMOE_MARK(u, MK_G_EPI_END);
   release_stage(ring_empty(R, use0));
   if (np > 1) release_stage(ring_empty(R, use0 + 1));
 }
@@ -1325,6 +1546,7 @@ __device__ __forceinline__ void dn_chunk(const Geo& G, const Chunk& c, const uin
   float acc[NR];
 #pragma unroll
   for (int i = 0; i < NR; ++i) acc[i] = 0.f;
+#pragma unroll 1
   for (int j = 0; j < G.ji; ++j) {
     const int s = lane_s + G.wi * j;
     const bool sok = s < G.si;
@@ -1354,6 +1576,57 @@ __device__ __forceinline__ void dn_chunk(const Geo& G, const Chunk& c, const uin
   });
 }
 
+// Stack layers after the first: x is the previous unit's output, read as its tagged words by
+// the 256 consumer threads (each word polled until it carries that unit's tag) into the x
+// buffer; the norm factor 1 / sqrt(mean(x^2) + eps) from a binary64 sum of squares taken in
+// the same order in every CTA; the owner CTA records x before the norm. While the words are
+// in flight, warp 0 also waits for every CTA's unit-done word of the previous unit: CTAs that
+// own no output rows write no words, and this keeps every CTA within one unit of the others
+// (the exchange buffers are reused every second unit). False (this warp) if a wait failed.
+__device__ __noinline__ bool fetch_x(const Prog& P, const Geo& G, Smem* sm,
+                                     const unsigned long long* xw, float* h_trace, int u,
+                                     float* XB, double* red) {
+  const int lane = threadIdx.x & 31;
+  const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
+  const int t = w * 32 + lane;
+  const unsigned long long want = tag32(u - 1);
+  bool bad = false;
+  double ss = 0.0;
+#pragma unroll 1
+  for (int b = 0; b < G.H; b += kConsumers * 16) {
+    unsigned long long v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = ld_relaxed_gpu_u64(xw + min(b + t + kConsumers * j, G.H - 1));
+    if (b == 0 && w == 0) bad = !warp_wait_done(P, sm, (unsigned)u, DE_TIMEOUT_DEP);
+    const int H = G.H;
+    if (!settle<16>(P, sm, v, [=](int j) { return xw + min(b + t + kConsumers * j, H - 1); },
+                    kTag32, want, DE_TIMEOUT_DEP))
+      bad = true;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int i = b + t + kConsumers * j;
+      if (i < G.H) {
+        const float x = value_of(v[j]);
+        XB[i] = x;
+        if (h_trace) h_trace[i] = x;
+        ss = fma((double)x, (double)x, ss);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[w] = ss;
+  consumers_sync();
+  if (t == 0) {
+    double a = 0.0;
+#pragma unroll
+    for (int q = 0; q < kConsumerWarps; ++q) a += red[q];
+    sm->xf[u & 1] = (float)(1.0 / sqrt(a / (double)G.H + (double)P.eps));
+  }
+  consumers_sync();
+  return !__any_sync(0xffffffffu, bad);
+}
+
 template <int BITS, int FORM, int NRG, int NRD>
 __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, const Share& S) {
   const int lane = threadIdx.x & 31;
@@ -1369,61 +1642,63 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
   unsigned a_used = 0, b_used = 0;  // chunks taken from each ring so far
   const int gslice = t % G.wh;           // this thread's x slice in gate/up rows
   const bool gu_on = G.shared_on || G.routed_on;
-  XRouter xr;
-  xr.seg = -1;
   // A wait that fails (its budget ran out, or the CTA aborted) marks the warp dead: it skips
   // every later wait but keeps walking the same sequence of chunks and consumer barriers as
   // the other warps, so that no warp is left at a barrier; the results are then undefined and
   // the error word reports the failure.
   bool dead = false;
   typename XOf<FORM>::T xg;              // x of this thread's slice (digits or values)
+#pragma unroll 1
   for (int u = 0; u < P.n_units; ++u) {
     const int slot_u = u & 1;
-    const UnitView uv = unit_view(P, G, u);
-    const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
-    if (!dead && !warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
+    if (P.mode == MODE_STACK && u % P.n_layers != 0) {
+      const UnitView uv = unit_view(P, G, u);
+      const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
+      if (!fetch_x(P, G, sm, uv.xw, owner ? uv.h_trace : nullptr, u, XB,
+                   reinterpret_cast<double*>(red)))
+        dead = true;
+    } else if (!dead && !warp_wait_ready(P, sm, &sm->x_ready, &sm->x_bar, (unsigned)(u + 1),
+                                         DE_TIMEOUT_DEP)) {
       dead = true;
+    }
+    if (t == 0 && !G.route_on) sm->sigma[slot_u] = 1.f;
     if (w == 0) FMOE_MARK(u, MK_K_X);
     // ---- router rows: whole rows in batches of up to kRouterBatch chunks, else chunk by chunk
-    if (G.route_on) {
-      if (S.nrc == 0) {
-        if (w == 0 && lane == 0 && !(P.debug & 1)) publish(P, SG_ROUTER, u);
-      } else if (G.rseg == 1 && G.rrows == 1) {
+    if (G.route_on && S.nrc > 0) {
+      if (G.rseg == 1 && G.rrows == 1) {
         const int bmax = min(kRouterBatch, A.ns);
+#pragma unroll 1
         for (int i0 = 0; i0 < S.nrc; i0 += bmax) {
           const int nb = min(bmax, S.nrc - i0);
+#pragma unroll 1
           for (int q = 0; q < nb; ++q) ring_wait(P, sm, A, a_used + (unsigned)q, dead);
-          if (xr.seg != 0) router_x(G, XB, 0, xr);
-          router_batch(P, G, sm, u, S.r0 + i0, nb, A, a_used, reinterpret_cast<double*>(red), xr,
-                       i0 + nb == S.nrc);
+          router_batch(P, G, sm, u, S.r0 + i0, nb, A, a_used, reinterpret_cast<double*>(red), XB);
           a_used += (unsigned)nb;
         }
       } else {
-        xr.seg = -1;
+#pragma unroll 1
         for (int i = 0; i < S.nrc; ++i) {
           const Chunk c = chunk_a(G, S, i);
           ring_wait(P, sm, A, a_used, dead);
-          if (xr.seg != c.seg) router_x(G, XB, c.seg, xr);
           router_chunk(P, G, sm, c, u, ring_stage(G, A, a_used), ring_empty(A, a_used),
-                       ring_slot(A, a_used), reinterpret_cast<double*>(red), xr, i == S.nrc - 1, 0u);
+                       ring_slot(A, a_used), reinterpret_cast<double*>(red), XB);
           ++a_used;
         }
       }
-      xr.seg = -1;  // the next unit's x differs
     }
     if (w == 0) FMOE_MARK(u, MK_K_ROUTER);
     // ---- x of this thread's slice: digit form (in place, after every router read of x)
     if (gu_on) {
-      consumers_sync();
-      const float xf = sm->xf[slot_u];
       if constexpr (FORM == FORM_DIGITS) {
-        transform<BITS>(XB, G.sh, xf);
+        consumers_sync();
+        transform<BITS>(XB, G.sh, sm->xf[slot_u]);
         consumers_sync();
         load_digits(XB, gslice < G.sh ? gslice : 0, xg);
       } else {
-        load_values(XB, gslice < G.sh ? gslice : 0, xf, xg);
+        consumers_sync();
+        load_values(XB, gslice < G.sh ? gslice : 0, sm->xf[slot_u], xg);
       }
-      // the x buffer is free once every warp holds its slice
+      // the x buffer and the digit form are free once every warp holds its slice
       if (lane == 0) {
         const unsigned old = atom_add_acq_rel_cta_smem(&sm->xd_arrive, 1u);
         if (old == (unsigned)(kConsumerWarps * (u + 1) - 1))
@@ -1432,49 +1707,60 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
       __syncwarp();
       if (w == 0) FMOE_MARK(u, MK_K_XD);
     }
-    // ---- routing decision: once every CTA's router rows of the unit are in
-    if (G.route_on) {
-      if (w == 0 && !dead &&
-          !warp_wait_sig(P, sm, SG_ROUTER, (unsigned)(u + 1), DE_TIMEOUT_ROUTE))
-        dead = true;
-      consumers_sync();
-      if (w == 0) FMOE_MARK(u, MK_C_S1);
-      topk_block(P, G, sm, u, P.s.logits + (size_t)slot_u * G.rseg * G.nr, uv.bias,
-                 owner ? uv.idx_out : nullptr, owner ? uv.w_out : nullptr);
-      consumers_sync();
-      if (w == 0) FMOE_MARK(u, MK_C_RT);
+    // ---- gate/up rows, in passes of up to gpass chunks: the shared expert (ring A) first,
+    // while the other CTAs' logits arrive; then the routing decision; then routed expert k
+    // (ring B) in turn
+    const int jobs = gu_on ? G.shared_on + (G.routed_on ? G.K : 0) : 0;
+#pragma unroll 1
+    for (int phase = 0; phase < 2; ++phase) {
+      if (phase == 1) {
+        // ---- routing decision: from every CTA's logit words of the unit, as they arrive
+        if (G.route_on) {
+          if (w == 0) FMOE_MARK(u, MK_C_S1);
+          const UnitView uv = unit_view(P, G, u);
+          const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
+          if (topk_block(P, G, sm, u, P.s.logits + (size_t)slot_u * G.rseg * G.nr, uv.bias,
+                         owner ? uv.idx_out : nullptr, owner ? uv.w_out : nullptr))
+            dead = true;
+          consumers_sync();
+          if (w == 0) FMOE_MARK(u, MK_C_RT);
+        }
+        if (G.nseg == 0 && t == 0) unit_done(P, u);  // no output rows: the unit ends here
+      }
+      const int j0 = phase == 0 ? 0 : G.shared_on;
+      const int j1 = phase == 0 ? min(G.shared_on, jobs) : jobs;
+#pragma unroll 1
+      for (int job = j0; job < j1; ++job) {
+        const bool sh = G.shared_on && job == 0;
+        const int k = job - G.shared_on;  // routed expert slot
+        if (w == 0 && k == 1) FMOE_MARK(u, MK_J1_TOP);
+        unsigned long long* hdst = P.s.hx + ((size_t)slot_u * G.nseg + job) * G.I;
+        const Ring R = sh ? A : B;
+        unsigned use = sh ? a_used : b_used;
+#pragma unroll 1
+        for (int i0 = 0; i0 < S.ngc; i0 += G.gpass) {
+          const int np = min(G.gpass, S.ngc - i0);
+          const Chunk c0 = sh ? chunk_a(G, S, S.nrc + i0) : chunk_b(G, S, k * S.ngc + i0);
+          const Chunk c1 = sh ? chunk_a(G, S, S.nrc + i0 + np - 1)
+                              : chunk_b(G, S, k * S.ngc + i0 + np - 1);
+          ring_wait(P, sm, R, use, dead);
+          if (w == 0 && k == 1 && i0 == 0) FMOE_MARK(u, MK_J1_W0);
+          if (np > 1) ring_wait(P, sm, R, use + 1, dead);
+          if (w == 0 && i0 == 0 && !sh) FMOE_MARK(u, MK_K_P2F + k);
+          gu_pass<BITS, FORM, NRG>(P, G, sm, np, c0, c1, R, use, red, xg, hdst, u,
+                                   !sh && k == 0 && i0 == 0);
+          use += (unsigned)np;
+        }
+        if (sh) a_used = use;
+        else b_used = use;
+        if (w == 0) FMOE_MARK(u, sh ? MK_K_SGU : MK_K_P2 + k);
+      }
     }
     if (!gu_on) continue;
-    // ---- gate/up rows: job 0 the shared expert (ring A), then routed expert k (ring B); each
-    // job in passes of up to gpass chunks
-    const int jobs = G.shared_on + (G.routed_on ? G.K : 0);
-    for (int job = 0; job < jobs; ++job) {
-      const bool sh = G.shared_on && job == 0;
-      const int k = job - G.shared_on;  // routed expert slot
-      const int sig = sh ? SG_SHARED : SG_EXP0 + k;
-      float* hdst = sh ? P.s.hs + (size_t)slot_u * G.I : P.s.hk + ((size_t)slot_u * G.K + k) * G.I;
-      const Ring R = sh ? A : B;
-      unsigned use = sh ? a_used : b_used;
-      if (S.ngc == 0 && w == 0 && lane == 0) publish(P, sig, u);
-      for (int i0 = 0; i0 < S.ngc; i0 += G.gpass) {
-        const int np = min(G.gpass, S.ngc - i0);
-        const Chunk c0 = sh ? chunk_a(G, S, S.nrc + i0) : chunk_b(G, S, k * S.ngc + i0);
-        const Chunk c1 = sh ? chunk_a(G, S, S.nrc + i0 + np - 1)
-                            : chunk_b(G, S, k * S.ngc + i0 + np - 1);
-        ring_wait(P, sm, R, use, dead);
-        if (np > 1) ring_wait(P, sm, R, use + 1, dead);
-        if (w == 0 && i0 == 0 && !sh) FMOE_MARK(u, MK_K_P2F + k);
-        gu_pass<BITS, FORM, NRG>(P, G, sm, np, c0, c1, R, use, red, xg, hdst, sig, u,
-                                 i0 + np == S.ngc);
-        use += (unsigned)np;
-      }
-      if (sh) a_used = use;
-      else b_used = use;
-      if (w == 0) FMOE_MARK(u, sh ? MK_K_SGU : MK_K_P2 + k);
-    }
     // ---- down rows: segment 0 the shared expert (ring A), then routed expert k (ring B), each
     // as soon as every CTA's h-rows of it are in; accumulated into this CTA's output rows
     if (S.ndc > 0) {
+#pragma unroll 1
       for (int sgm = 0; sgm < G.nseg; ++sgm) {
         const bool sh = G.shared_on && sgm == 0;
         const int k = sgm - G.shared_on;
@@ -1492,6 +1778,7 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
         }
         const Ring R = sh ? A : B;
         unsigned use = sh ? a_used : b_used;
+#pragma unroll 1
         for (int i = 0; i < S.ndc; ++i) {
           const Chunk c = sh ? chunk_a(G, S, S.nrc + S.ngc + i)
                              : chunk_b(G, S, G.K * S.ngc + k * S.ndc + i);
@@ -1509,20 +1796,18 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
     if (G.nseg > 0) {
       if (S.d1 > S.d0) consumers_sync();
       if (w == 0) {
-        float sq = 0.f;
+        const UnitView uv = unit_view(P, G, u);  // (recomputed: not held through the unit)
+#pragma unroll 1
         for (int r = S.d0 + lane; r < S.d1; r += 32) {
-          const float o = (uv.res ? __ldcg(uv.res + r) : 0.f) + oacc[r - S.d0];
+          const float res = uv.resw ? value_of(__ldcg(uv.resw + r))
+                                    : (uv.res ? __ldcg(uv.res + r) : 0.f);
+          const float o = res + oacc[r - S.d0];
           oacc[r - S.d0] = 0.f;
-          uv.out[r] = o;
-          sq += o * o;
-        }
-        if (P.mode == MODE_STACK && S.d1 > S.d0) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-          if (lane == 0) atomicAdd(P.s.normsq + u, sq);
+          if (uv.outw) st_relaxed_gpu_u64(uv.outw + r, value_word(o, u));
+          else uv.out[r] = o;
         }
         __syncwarp();
-        if (lane == 0) publish(P, SG_OUT, u);
+        if (lane == 0) unit_done(P, u);
         FMOE_MARK(u, MK_K_OUT);
       }
     }
@@ -1537,20 +1822,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G.o_bar);
   if (threadIdx.x == 0) {
     sm->abort = 0;
-    sm->x_ready = sm->rt_ready = sm->hs_ready = sm->hk_ready = sm->xfree = 0;
+    sm->x_ready = sm->rt_ready = sm->hs_ready = sm->hk_ready = sm->xfree = sm->gu_issued = 0;
     sm->xd_arrive = 0;
+#pragma unroll 1
     for (int i = 0; i < 2 * kMaxStages; ++i) sm->chunk_arrive[i] = 0;
     mbar_init(&sm->xbar, 1);
-    mbar_init(&sm->hbar, 1);
     mbar_init(&sm->x_bar, 1);
     mbar_init(&sm->rt_bar, 1);
     mbar_init(&sm->hs_bar, 1);
     mbar_init(&sm->hk_bar, 1);
     mbar_init(&sm->xfree_bar, 1);
+#pragma unroll 1
     for (int i = 0; i < G.nA; ++i) {
       mbar_init(&bars[i], 1);
       mbar_init(&bars[G.nA + i], kConsumerWarps);
     }
+#pragma unroll 1
     for (int i = 0; i < G.nB; ++i) {
       mbar_init(&bars[2 * G.nA + i], 1);
       mbar_init(&bars[2 * G.nA + G.nB + i], kConsumerWarps);
@@ -1558,16 +1845,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   float* oacc = reinterpret_cast<float*>(smem + G.o_oacc);
+#pragma unroll 1
   for (int i = threadIdx.x; i < G.oacc_n; i += blockDim.x) oacc[i] = 0.f;
   __syncthreads();
   const Share S = make_share(G);
   const int warp = threadIdx.x >> 5;
   if (warp == 0) {
-    producer_a(P, G, smem, sm, S);
+    if ((threadIdx.x & 31) == 0) producer_a(P, G, smem, sm, S);
   } else if (warp == 1) {
-    producer_b(P, G, smem, sm, S);
+    if ((threadIdx.x & 31) == 0) producer_b(P, G, smem, sm, S);
   } else if (warp == 2) {
-    controller(P, G, smem, sm);
+    controller(P, G, smem, sm, S.ndc > 0);
   } else {
     consumer<BITS, FORM, kMaxRowsThread, kMaxRowsWarp>(P, G, smem, sm, S);
   }

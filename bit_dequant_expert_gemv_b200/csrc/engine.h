@@ -16,10 +16,17 @@
 //          (expert k = 0..K-1 in turn), then their down chunks.
 // The consumer warps work through a unit in the order
 //   router (A) -> shared gate/up (A) -> shared down (A) -> routed gate/up k (B) -> routed down k (B)
-// with every warp taking part in every chunk. Cross-CTA dependencies are counted on monotone
-// global counters (one per signal, each on its own 128-byte line): a CTA adds the number of
-// rows it finished; signal s of unit u is complete when every CTA's word for s has reached
-// u + 1 (each CTA publishes its own progress word; no two CTAs write the same word).
+// with every warp taking part in every chunk.
+// Cross-CTA data moves as self-validating 64-bit words, written without fences and read by
+// polling: each word carries the unit it belongs to (a tag), so a reader that sees the right
+// tag has the value, and no flag, release fence or second round trip is needed:
+//   router logits   binary64, the tag in the 13 lowest mantissa bits;
+//   h values        {binary32 value, 32-bit tag};
+//   stack outputs   {binary32 value, 32-bit tag} (the next layer's input).
+// Where nothing is read (one token's output before an independent next token), each CTA
+// stores a per-CTA "unit done" word instead, and the next unit starts once every CTA's word
+// shows the previous unit. Every exchange buffer is zeroed before each launch; tags are never
+// zero.
 #pragma once
 #include <stdint.h>
 
@@ -31,24 +38,17 @@ constexpr int kCtrlWarps = 3;                      // producer A, producer B, co
 constexpr int kThreads = kConsumers + 32 * kCtrlWarps;
 constexpr int kMaxLayers = 128;
 constexpr int kMaxK = 8;
-constexpr unsigned kStage = 18432;                 // bytes per ring stage
+constexpr unsigned kStage = 36864;                 // bytes per ring stage
 constexpr int kRouterCols = 4 * 4 * 256;           // router columns per chunk (4 float4 per thread)
 constexpr int kMaxStages = 16;                     // per ring
 constexpr int kMaxRowsThread = 8;                  // gate/up rows one consumer thread holds
 constexpr int kMaxRowsWarp = 4;                    // down rows (per side-by-side lane group) a warp holds
 constexpr int kMaxHr = 64;                         // h-rows per gate/up chunk (cap)
 
-// Global signals: per signal one progress word per CTA (Scratch::ctrl[s * kMaxCtas + cta]),
-// the number of units whose rows of that phase the CTA has finished.
-enum Sig {
-  SG_ROUTER = 0,   // router rows finished (logits written)
-  SG_SHARED = 1,   // shared-expert h-rows finished
-  SG_OUT = 2,      // output rows finished (out written, sum of squares added)
-  SG_EXP0 = 3,     // + k: routed expert k's h-rows finished
-  SG_COUNT = SG_EXP0 + kMaxK
-};
+// Per-CTA "unit done" words (Scratch::ctrl[cta]): the number of units whose output rows the
+// CTA has written.
 constexpr int kMaxCtas = 256;                      // grid size limit (one CTA per SM)
-constexpr int kCtrlWords = kMaxCtas * SG_COUNT;
+constexpr int kCtrlWords = kMaxCtas;
 constexpr int kMiscBytes = 4096;                   // small shared state (Smem)
 
 enum ModeBits { MODE_SEQ = 0, MODE_STACK = 1 };
@@ -94,14 +94,13 @@ struct Geo {
   unsigned smem_bytes;
 };
 
+// Exchange buffers, indexed by unit parity; all zeroed before each launch.
 struct Scratch {
-  unsigned* ctrl;        // kCtrlWords progress words, zeroed per launch
-  int* err;              // sticky per-device error word
-  double* logits;        // [2][rseg][nr] per unit parity: partial logits per column segment
-  float* hs;             // [2][I]
-  float* hk;             // [2][K][I]
-  float* normsq;         // [n_units], zeroed per launch
-  float* hbuf;           // [2][H]
+  unsigned* ctrl;                 // kCtrlWords unit-done words
+  int* err;                       // sticky per-device error word
+  unsigned long long* logits;     // [2][rseg][nr] tagged binary64 partial logits per column segment
+  unsigned long long* hx;         // [2][nseg][I] tagged h values: shared expert first, then routed k
+  unsigned long long* hbuf;       // [2][H] tagged stack outputs (STACK mode only; else null)
 };
 
 struct Prog {

@@ -267,19 +267,19 @@ uint64_t fmoe_launch_count(void);
  * the device).
  *
  * Same arguments, layout, validation and result as fmoe_moe_layer (one token). The library
- * scratch of the call (phase counters, router logits, h vectors) lives in
+ * scratch of the call (unit-done words, tagged router logits, tagged h vectors) lives in
  * one fixed device array of FMOE_NOALLOC_SCRATCH_BYTES per device, compiled into the library;
  * the call makes no cudaMalloc, cudaFree, pool or other allocating call.
  *   - The first call on a device does the setup: it obtains the array's address with
  *     cudaGetSymbolAddress (which also loads the library's kernels on that device), zeroes the
  *     array's error word and sets the kernel's shared-memory limit. Make that first call with
  *     the device current and outside any stream capture; later calls only enqueue work.
- *   - The phase counters must start at zero for every launch: each call zeroes them with
- *     cudaMemsetAsync on `stream` before its launch. Nothing else needs zeroing.
+ *   - The exchange words must start at zero for every launch: each call zeroes the scratch
+ *     it uses with one cudaMemsetAsync on `stream` before its launch.
  *   - Shapes whose scratch exceeds the array (beyond FMOE_NOALLOC_SCRATCH_BYTES minus 256
  *     bytes for the error word; e.g. 4096 experts with top_k = 8 and I = 1024) return
  *     FMOE_ERR_UNSUPPORTED with the needed size in fmoe_last_error(); nothing is enqueued.
- *     The full-size layer (H = 4096, I = 1024, E = 512, K = 4) needs about 90 KB.
+ *     The full-size layer (H = 4096, I = 1024, E = 512, K = 4) needs 91,392 bytes.
  *   - There is one array per device: two calls of this function on one device whose work can
  *     overlap (different streams, or host threads without ordering) race on it and give
  *     undefined results. Calls on one stream are ordered and safe.

@@ -140,11 +140,22 @@ def test_layer_full_q4_forced_bench_launch(fmoe, orc):
     out, idx, w, x, res = run_seq(fmoe, wl, T, bias=bias, replicas=4)
     forced = synth.forced_experts(wl, tokens=T)[:, 0]
     assert all(set(idx[t].tolist()) == set(forced[t].tolist()) for t in range(T))
-    check_tokens(orc, wl, [0, 1, 517, T - 1], out, idx, w, x, res, bias=bias)
+    check_tokens(orc, wl, sample_tokens(T, 32, seed=5), out, idx, w, x, res, bias=bias)
     assert np.isfinite(out).all()
 
 
+def sample_tokens(T, n, seed):
+    """The first and last token and n - 2 others drawn without replacement (seeded)."""
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
+    return [0, *sorted(int(t) for t in mid), T - 1]
+
+
 def test_layer_full_q2(fmoe, orc):
+    """The 2-bit layer's whole token sequence (1000 tokens, natural routing) in one launch;
+    32 sampled tokens against the oracle."""
     wl = synth.WORKLOADS["full_q2"]
-    out, idx, w, x, res = run_seq(fmoe, wl, 5)
-    check_tokens(orc, wl, [0, 4], out, idx, w, x, res)
+    T = wl.tokens
+    out, idx, w, x, res = run_seq(fmoe, wl, T)
+    check_tokens(orc, wl, sample_tokens(T, 32, seed=6), out, idx, w, x, res)
+    assert np.isfinite(out).all()

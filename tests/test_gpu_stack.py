@@ -7,7 +7,7 @@ import torch
 
 import synth
 from oracle.workload import HostLayer
-from gpu_helpers import check_out, check_routing, renorm_weights
+from gpu_helpers import ABS_TOL, REL_L2, check_out, check_routing, renorm_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -102,6 +102,35 @@ def test_stack_full_size(fmoe, orc, name):
                 assert set(idx[t, l].tolist()) == set(forced[t, l].tolist())
     L = wl.layers
     pairs = [(0, 0), (0, 1), (1, L // 2), (2, L - 1)]
-    teacher_force(orc, wl, {}, pairs, h_in, idx, ht, h_out, bias=bias)
+    hls = {}
+    teacher_force(orc, wl, hls, pairs, h_in, idx, ht, h_out, bias=bias)
+    if name != "stack_q4_skewed":
+        end_to_end(orc, wl, hls, 0, h_in, idx, h_out, bias=bias)
     del dls
     torch.cuda.empty_cache()
+
+
+def end_to_end(orc, wl, hls, t, h_in, idx, h_out, bias=None):
+    """Token t through every layer by the oracle alone, from the same input: the oracle's own
+    chain of h, not the GPU's recorded layer inputs. The selection is the oracle's wherever it
+    is unambiguous; inside the tie band the chain takes the GPU's (both are correct there),
+    so that the two chains stay comparable. The per-layer bounds hold for one layer; over a
+    chain each layer adds its own rounding error to the residual stream, and independent
+    errors grow like the square root of the depth: the end-to-end output is held to the same
+    relative-L2 bound (1e-3) and to max-abs <= 2e-3 * sqrt(L). Its error is reported."""
+    L = wl.layers
+    h = h_in[t].astype(np.float64)
+    for l in range(L):
+        hl = hls.setdefault(l, HostLayer(orc, wl, l))
+        x = h if l == 0 else orc.rmsnorm(h, wl.eps)
+        bb = None if bias is None else bias[t, l]
+        oi, ow, logits, _ = orc.route(x, hl.router, bb, wl.K)
+        if check_routing(idx[t, l], None, logits, wl.K):
+            h = hl.forced(x, h, oi, ow)
+        else:
+            h = hl.forced(x, h, idx[t, l], renorm_weights(logits, idx[t, l]))
+    got, want = h_out[t].astype(np.float64), h
+    err = np.abs(got - want).max()
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    print(f"{wl.name} token {t}, {L} layers end to end: max-abs {err:.3e}, rel-L2 {rel:.3e}")
+    assert err <= ABS_TOL * np.sqrt(L) and rel <= REL_L2, (wl.name, t, err, rel)
