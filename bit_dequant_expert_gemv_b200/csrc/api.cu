@@ -222,8 +222,9 @@ int make_geo(int H, int I, int E, int K, int bits, bool route_on, bool shared_on
   // reads x, read by the consumers before any h value arrives)
   const unsigned h_b = std::max(4u * (unsigned)(G->nseg * I), x_b);
   const unsigned wn = G->wh > 32 ? (unsigned)G->wh / 32 : 1u;
-  const unsigned red_slot = std::max(8u * (unsigned)G->rrows * kConsumerWarps,
-                                     4u * 2u * (unsigned)(G->gpass * G->hr) * wn);
+  const unsigned red_slot =
+      std::max(8u * (unsigned)std::max(G->rrows, kRouterBatch) * kConsumerWarps,
+               4u * 2u * (unsigned)(G->gpass * G->hr) * wn);
   const unsigned oacc_b = 4u * (unsigned)std::max(G->oacc_n, 1);
   const unsigned misc_b = kMiscBytes;
   const unsigned fixed = align_up(x_b, 128) + align_up(std::max(h_b, 128u), 128) +

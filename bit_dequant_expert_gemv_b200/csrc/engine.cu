@@ -83,7 +83,6 @@ struct Smem {
   unsigned hs_ready;           // units whose h_s is in the h buffer
   unsigned hk_ready;           // routed segments ready, counted over units: u*K + k + 1
   unsigned xfree;              // units whose x buffer the consumers no longer read
-  unsigned gu_issued;          // units whose routed gate/up copies producer B has all issued
   unsigned xd_arrive;          // consumer warps done loading x digits (8 per unit)
   unsigned chunk_arrive[2 * kMaxStages];  // per stage (ring A, then B): warps done with it
   float xf[2];                 // RMSNorm factor of the unit's x (1 without a norm)
@@ -581,44 +580,6 @@ __device__ void drain_ring(const Prog& P, uint64_t* full, int ns, unsigned issue
   }
 }
 
-// Request chunks [i0, i1) of ring B's list for the unit routed to `rte` into L2 (one thread).
-__device__ __forceinline__ void prefetch_chunks_b(const Geo& G, const Share& S, const LayerW& L,
-                                                  const int* rte, int i0, int i1) {
-#pragma unroll 1
-  for (int i = i0; i < i1; ++i) {
-    const Chunk c = chunk_b(G, S, i);
-    const int e = min(max(rte[c.e], 0), G.E - 1);
-    const uint8_t* eb = L.experts + (size_t)e * L.expert_stride;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint8_t* src = nullptr;
-      unsigned dst_off = 0;
-      const unsigned bytes = copy_desc(G, L, eb, c, q, &src, &dst_off);
-      if (bytes) prefetch_l2_bulk(src, bytes);
-    }
-  }
-}
-
-// One thread: wait until the shared-memory counter *cnt reaches target (wrap-safe), bounded
-// like every other wait.
-__device__ __noinline__ bool wait_ready_counter(const Prog& P, Smem* sm, const unsigned* cnt,
-                                                unsigned target, int code) {
-  if ((int)(ld_acquire_cta_smem(cnt) - target) >= 0) return true;
-  const uint64_t deadline = global_ns() + P.wait_ns;
-#pragma unroll 1
-  for (unsigned it = 0;; ++it) {
-    __nanosleep(64);
-    if ((int)(ld_acquire_cta_smem(cnt) - target) >= 0) return true;
-    if ((it & 7) == 7) {
-      if (sm->abort) return false;
-      if (global_ns() > deadline) {
-        raise_error(P, sm, code);
-        return false;
-      }
-    }
-  }
-}
-
 // Producers run on one thread each (lane 0 of warps 0 and 1; the other lanes have left).
 __device__ void producer_a(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
                            const Share& S) {
@@ -626,17 +587,9 @@ __device__ void producer_a(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
   uint64_t* empty = full + G.nA;
   unsigned issued = 0;
   bool failed = false;
-  const bool gate = G.routed_on && S.nb > 0;
 #pragma unroll 1
   for (int u = 0; u < P.n_units && !failed; ++u) {
     const LayerW& L = P.layers[u % P.n_layers];
-    // The next unit's data-independent rows wait until the previous unit's routed gate/up
-    // copies are all out: they are needed later, and would otherwise share HBM with the
-    // stream that decides how soon the previous unit's gate/up rows are done.
-    if (gate && u > 0 && !wait_ready_counter(P, sm, &sm->gu_issued, (unsigned)u, DE_TIMEOUT_DEP)) {
-      failed = true;
-      break;
-    }
 #pragma unroll 1
     for (int i = 0; i < S.na; ++i) {
       const Chunk c = chunk_a(G, S, i);
@@ -670,18 +623,8 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
     }
     FMOE_MARK(u, MK_B_RT);
     const int* rte = sm->rt_e[u & 1];
-    // The first ring-full of chunks goes out first; then the gate/up copies that the ring
-    // cannot take yet are requested into L2 (so that HBM streams the CTA's whole routed
-    // gate/up share at once and the ring's later copies hit L2); the down copies follow the
-    // same way once every gate/up copy is out.
-    const int ngu = G.K * S.ngc;
 #pragma unroll 1
     for (int i = 0; i < S.nb; ++i) {
-      if (i == min(G.nB, ngu)) prefetch_chunks_b(G, S, L, rte, i, ngu);
-      if (i == ngu) {
-        st_release_cta_smem(&sm->gu_issued, (unsigned)(u + 1));
-        prefetch_chunks_b(G, S, L, rte, max(i, G.nB), S.nb);
-      }
       const Chunk c = chunk_b(G, S, i);
       const int e = min(max(rte[c.e], 0), G.E - 1);
       const uint8_t* eb = L.experts + (size_t)e * L.expert_stride;
@@ -696,7 +639,6 @@ __device__ void producer_b(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
       if (i == 3) FMOE_MARK(u, MK_B_I3);
       ++issued;
     }
-    if (ngu == S.nb) st_release_cta_smem(&sm->gu_issued, (unsigned)(u + 1));
   }
   if (failed) drain_ring(P, full, G.nB, issued);
 }
@@ -1103,6 +1045,7 @@ __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
     if (G.route_on && uv.bias)  // the unit's logit bias into L2 while the router runs
 #pragma unroll 1
       for (int e = lane * 32; e < G.E; e += 32 * 32) prefetch_l2(uv.bias + e);
+
     // ---- independent tokens: the next unit's x, once the consumers hold this unit's x
     // digits in registers (its computation still waits for this unit to complete)
     if (P.mode == MODE_SEQ && x_digits && u + 1 < P.n_units) {
@@ -1363,19 +1306,26 @@ __device__ __forceinline__ double row_dot4(const float4* ws, int f, const X4& x,
   return fma((double)wv.w, x.d, acc);
 }
 
-// Whole router rows, one per chunk, of up to kRouterBatch consecutive chunks at once: each
-// thread takes float4 columns t + 512 j of every row, with an independent binary64 chain per
-// (row, j); one transposing warp reduction for all rows; the warp partials through shared
-// memory, summed in warp order by the batch's last warp, which stores the logits.
-constexpr int kRouterBatch = 4;
-
+// Whole router rows, up to kRouterBatch of them from consecutive chunks of G.rrows rows each
+// (row r of the batch is row r % rrows of chunk use0 + r / rrows): each thread takes float4
+// columns t + 256 j of every row, x converted once per column group, one independent binary64
+// chain per row; one transposing warp reduction for all rows; the warp partials through
+// shared memory, summed in warp order by the batch's last warp, which stores the logits.
 __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* sm, int u,
-                                             int r0, int nrows, const Ring& R, unsigned use0,
-                                             double* red, const float* XB) {
+                                             int r0, int nrows, int nchunks, const Ring& R,
+                                             unsigned use0, double* red, const float* XB) {
   const int lane = threadIdx.x & 31;
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
   const int t = w * 32 + lane;
   const int nf = G.rcols / 4;
+  const float4* ws[kRouterBatch];
+#pragma unroll
+  for (int r = 0; r < kRouterBatch; ++r) {
+    const int rr = r < nrows ? r : 0;
+    const int q = rr / G.rrows;
+    ws[r] = reinterpret_cast<const float4*>(ring_stage(G, R, use0 + (unsigned)q)) +
+            (size_t)(rr - q * G.rrows) * nf;
+  }
   double v[kRouterBatch];
 #pragma unroll
   for (int r = 0; r < kRouterBatch; ++r) v[r] = 0.0;
@@ -1385,11 +1335,8 @@ __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* 
     if (f < nf) {
       const X4 x = router_x4(G, XB, 0, f);
 #pragma unroll
-      for (int r = 0; r < kRouterBatch; ++r) {
-        const float4* ws = reinterpret_cast<const float4*>(
-            ring_stage(G, R, use0 + (unsigned)(r < nrows ? r : 0)));
-        if (r < nrows) v[r] = row_dot4(ws, f, x, v[r]);
-      }
+      for (int r = 0; r < kRouterBatch; ++r)
+        if (r < nrows) v[r] = row_dot4(ws[r], f, x, v[r]);
     }
   }
   FMOE_MARK_W(u, MK_R_DOT, MK_R_DOT_W);
@@ -1413,7 +1360,7 @@ __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* 
     FMOE_MARK(u, MK_R_PUB);
   }
 #pragma unroll 1
-  for (int r = 0; r < nrows; ++r) release_stage(ring_empty(R, use0 + (unsigned)r));
+  for (int q = 0; q < nchunks; ++q) release_stage(ring_empty(R, use0 + (unsigned)q));
 }
 
 __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* sm,
@@ -1663,17 +1610,19 @@ __device__ void consumer(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm, c
     }
     if (t == 0 && !G.route_on) sm->sigma[slot_u] = 1.f;
     if (w == 0) FMOE_MARK(u, MK_K_X);
-    // ---- router rows: whole rows in batches of up to kRouterBatch chunks, else chunk by chunk
+    // ---- router rows: whole rows in batches of up to kRouterBatch rows, else chunk by chunk
     if (G.route_on && S.nrc > 0) {
-      if (G.rseg == 1 && G.rrows == 1) {
-        const int bmax = min(kRouterBatch, A.ns);
+      if (G.rseg == 1 && G.rrows <= kRouterBatch) {
+        const int cmax = max(1, min(kRouterBatch / G.rrows, A.ns));  // chunks per batch
 #pragma unroll 1
-        for (int i0 = 0; i0 < S.nrc; i0 += bmax) {
-          const int nb = min(bmax, S.nrc - i0);
+        for (int i0 = 0; i0 < S.nrc; i0 += cmax) {
+          const int nc = min(cmax, S.nrc - i0);
 #pragma unroll 1
-          for (int q = 0; q < nb; ++q) ring_wait(P, sm, A, a_used + (unsigned)q, dead);
-          router_batch(P, G, sm, u, S.r0 + i0, nb, A, a_used, reinterpret_cast<double*>(red), XB);
-          a_used += (unsigned)nb;
+          for (int q = 0; q < nc; ++q) ring_wait(P, sm, A, a_used + (unsigned)q, dead);
+          const int rb = S.r0 + i0 * G.rrows;
+          router_batch(P, G, sm, u, rb, min(nc * G.rrows, S.r1 - rb), nc, A, a_used,
+                       reinterpret_cast<double*>(red), XB);
+          a_used += (unsigned)nc;
         }
       } else {
 #pragma unroll 1
@@ -1822,7 +1771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G.o_bar);
   if (threadIdx.x == 0) {
     sm->abort = 0;
-    sm->x_ready = sm->rt_ready = sm->hs_ready = sm->hk_ready = sm->xfree = sm->gu_issued = 0;
+    sm->x_ready = sm->rt_ready = sm->hs_ready = sm->hk_ready = sm->xfree = 0;
     sm->xd_arrive = 0;
 #pragma unroll 1
     for (int i = 0; i < 2 * kMaxStages; ++i) sm->chunk_arrive[i] = 0;

@@ -44,6 +44,7 @@ constexpr int kMaxStages = 16;                     // per ring
 constexpr int kMaxRowsThread = 8;                  // gate/up rows one consumer thread holds
 constexpr int kMaxRowsWarp = 4;                    // down rows (per side-by-side lane group) a warp holds
 constexpr int kMaxHr = 64;                         // h-rows per gate/up chunk (cap)
+constexpr int kRouterBatch = 4;                    // router rows reduced together
 
 // Per-CTA "unit done" words (Scratch::ctrl[cta]): the number of units whose output rows the
 // CTA has written.

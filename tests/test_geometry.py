@@ -133,6 +133,8 @@ def check_reads(G, kind, r0, n, seg, cov, d0):
                 assert inside(cov, (r * nf + f) * 16, 16), (r, f)
             assert (seg * cols + 4 * (nf - 1) + 4) <= G["H"]
         assert (n * WARPS) * 8 <= G["red_slot"]
+        if G["rseg"] == 1 and G["rrows"] <= 4:  # batches of up to 4 rows across chunks
+            assert (4 * WARPS) * 8 <= G["red_slot"]
         return
     if kind == CK_GU:
         NR = G["max_rows_thread"]
