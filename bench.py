@@ -34,6 +34,10 @@ REPLICAS = 16
 # as three signed 8-bit digit planes, integer dp4a products, fp32 combine and accumulation;
 # router dot products are fp32 x fp32 accumulated in binary64.
 DTYPE = "u4/u2 x s8x3-digit dp4a -> fp32 (router f32->f64)"
+# the arithmetic of each selectable dot-product form (fmoe_set_dot_form)
+FORMS = {"digits": (0, DTYPE),
+         "fma": (1, "u4/u2 -> f32, fma(q, s*x, z*x) per weight -> fp32 (router f32->f64)"),
+         "naive": (2, "u4/u2 -> f32, (q*s + z)*x per weight -> fp32 (router f32->f64)")}
 
 
 def parse():
@@ -51,6 +55,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--form", default="digits", choices=sorted(FORMS),
+                    help="dot-product form of the expert GEMVs (the pages' FMA comparison)")
     return ap.parse_args()
 
 
@@ -69,7 +75,7 @@ def max_over_ranks(value: float, device, world: int) -> float:
     return float(t.item())
 
 
-def arm_config(wl, T: int, world: int) -> dict:
+def arm_config(wl, T: int, world: int, form: str = "digits") -> dict:
     """The `config` object of the JSON line; both arms report the same one."""
     stack = wl.layers > 1
     return {"workload": wl.name, "hidden": wl.H, "experts": wl.E, "top_k": wl.K,
@@ -79,7 +85,8 @@ def arm_config(wl, T: int, world: int) -> dict:
             "l2": ("inputs larger than L2: 16 round-robin copies of router/shared expert, "
                    "512 routed experts (3.6 GB)") if not stack else
                   "inputs larger than L2: every layer's tensors once per token",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "dot_form": form}
 
 
 def peaks():
@@ -265,7 +272,7 @@ def run_reference(args):
             "ms_per_step": 1000.0 * statistics.median(secs), "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": arm_config(wl0, args.tokens or wl0.tokens, world),
+            "config": arm_config(wl0, args.tokens or wl0.tokens, world, args.form),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -289,6 +296,7 @@ def run_ours(args):
     import synth
     from bit_dequant_expert_gemv_b200.workload import build_layer, token_inputs_dev
     fmoe.build()
+    fmoe.set_dot_form(FORMS[args.form][0])
 
     wl = synth.WORKLOADS[args.workload]
     if args.experts:
@@ -404,8 +412,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": DTYPE, "data": "synthetic",
-            "config": arm_config(wl, T, world),
+            "dtype": FORMS[args.form][1], "data": "synthetic",
+            "config": arm_config(wl, T, world, args.form),
             "us_per_layer": ms_per_step * 1000.0 / layers_per_step,
             "gbs_algorithmic": bytes_per_layer * layers_per_step / (ms_per_step / 1000.0) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
