@@ -41,8 +41,8 @@
 #include "engine.h"
 #include "ptx.cuh"
 
-// Timeline hooks (a point of a unit's progress reached by one role), used by an external
-// profiling build; they expand to nothing in the library.
+// Timeline hooks (a point of a unit's progress reached by one role), defined by the profiling
+// build of timeline/timeline.py (timeline/marks.cuh); they expand to nothing in the library.
 #ifndef FMOE_MARK
 #define FMOE_MARK(u, ev) ((void)0)
 #endif
