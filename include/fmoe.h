@@ -25,6 +25,10 @@
  *     last failure on the calling host thread is in fmoe_last_error().
  *   - Errors raised inside a kernel (a bounded wait that ran out) are sticky per device and
  *     are read with fmoe_sync_status().
+ *   - The layer entry points run one persistent kernel with one CTA per SM whose CTAs wait
+ *     on each other; it is launched cooperatively, so a launch whose CTAs cannot all be
+ *     resident at once (another kernel holding SMs, MPS limits) fails at launch with
+ *     FMOE_ERR_CUDA instead of waiting out its budget.
  *   - Device pointers to packed weights, activations and outputs must be 16-byte aligned
  *     (FMOE_ERR_ALIGN otherwise).
  *   - Shapes: hidden H and intermediate I are multiples of 64 with 64 <= H,I <= 8192;
@@ -96,9 +100,9 @@ int fmoe_sync_status(void* stream);
 void fmoe_set_wait_budget_ns(uint64_t ns);
 
 /* Test hook: bit 0 makes every kernel launched afterwards on the calling host thread compute
- * but never publish its routing decision, so every wait that depends on it runs out of its
- * budget and the launch ends with FMOE_ERR_TIMEOUT (a host-made failure for testing the
- * timeout path; nothing faults). 0 restores normal operation. */
+ * its router logits but never write them for the other CTAs, so every wait that depends on
+ * them runs out of its budget and the launch ends with FMOE_ERR_TIMEOUT (a host-made failure
+ * for testing the timeout path; nothing faults). 0 restores normal operation. */
 void fmoe_set_fault_injection(int flags);
 
 /* ---------------------------------------------------------------------------------------
