@@ -761,15 +761,10 @@ __device__ __noinline__ bool topk_block(const Prog& P, const Geo& G, Smem* sm, i
   const int w = ((int)threadIdx.x >> 5) - kCtrlWarps;
   bool bad = false;
   float gate_l = 0.f;
-  if (w == 0 && lane == 0 && G.gate_on) {  // the shared-gate row's logit (sigma), early
-    double a = 0.0;
-#pragma unroll 1
-    for (int sg = 0; sg < G.rseg; ++sg) {
-      const size_t at = (size_t)sg * G.nr + G.E;
-      a += logit_part(P, sm, lg, ld_relaxed_gpu_u64(lg + at), at, u, bad);
-    }
-    gate_l = (float)a;
-  }
+  // the shared-gate row's logit (sigma): its first word is loaded now, with the experts' words
+  // below in flight beside it, and settled after them
+  const bool gate_lane = w == 0 && lane == 0 && G.gate_on;
+  const unsigned long long gate_w0 = gate_lane ? ld_relaxed_gpu_u64(lg + G.E) : 0ull;
   unsigned long long best_key = 0ull;  // lane k < K: the warp's k-th best so far
   double best_l = 0.0;
   constexpr int kBlock = 64 * kConsumerWarps;
@@ -827,6 +822,16 @@ __device__ __noinline__ bool topk_block(const Prog& P, const Geo& G, Smem* sm, i
       lv[1] = bl;
       warp_topk<2>(G.K, key, lv, best_key, best_l);
     }
+  }
+  if (gate_lane) {
+    double a = 0.0;
+    a += logit_part(P, sm, lg, gate_w0, (size_t)G.E, u, bad);
+#pragma unroll 1
+    for (int sg = 1; sg < G.rseg; ++sg) {
+      const size_t at = (size_t)sg * G.nr + G.E;
+      a += logit_part(P, sm, lg, ld_relaxed_gpu_u64(lg + at), at, u, bad);
+    }
+    gate_l = (float)a;
   }
   bad = __any_sync(0xffffffffu, bad);
   if (lane < G.K) {
@@ -1057,10 +1062,16 @@ __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
     const UnitView uv = unit_view(P, G, u);
     const bool owner = (u % (int)gridDim.x) == (int)blockIdx.x;
     FMOE_MARK(u, MK_C_UNIT);
-    // ---- x(u) from an input buffer: computed on only after unit u-1 is done everywhere
-    // (stack layers after the first read the previous layer's words in the consumers)
+    // ---- x(u) from an input buffer. Independent tokens with expert rows: unit u starts once
+    // every CTA has finished unit u-2 (the logit and h buffers alternate between units and
+    // every word carries its unit, so a CTA one unit ahead overwrites only words of unit u-2,
+    // which no CTA reads any more; this CTA's x buffer is refilled only after its consumers
+    // freed it). Otherwise (router only, whose x copy nothing else orders after the
+    // consumers' reads; a stack's first layer) once unit u-1 is done everywhere. Stack layers
+    // after the first read the previous layer's words in the consumers.
     if (uv.xin) {
-      if (u > 0 && !warp_wait_done(P, sm, (unsigned)u, DE_TIMEOUT_DEP)) break;
+      const int lag = P.mode == MODE_SEQ && x_digits ? 2 : 1;
+      if (u >= lag && !warp_wait_done(P, sm, (unsigned)(u + 1 - lag), DE_TIMEOUT_DEP)) break;
       FMOE_MARK(u, MK_C_PREV_DONE);
       if (!x_issued) copy_in(XB, uv.xin, 4u * (unsigned)G.H, &sm->xbar);
       x_issued = false;
@@ -1090,6 +1101,10 @@ __device__ void controller(const Prog& P, const Geo& G, uint8_t* smem, Smem* sm,
       x_issued = true;
     }
     if (G.nseg == 0 || !need_h) continue;  // (no output rows: no h needed)
+    // the h buffer is refilled only after this CTA's consumers have left unit u-1 (they hold
+    // unit u's x): without a router nothing else orders the two
+    if (!warp_wait_ready(P, sm, &sm->xfree, &sm->xfree_bar, (unsigned)(u + 1), DE_TIMEOUT_DEP))
+      break;
     // ---- h of unit u, segment by segment (shared expert, then routed k), as its words arrive
     bool ok = true;
 #pragma unroll 1

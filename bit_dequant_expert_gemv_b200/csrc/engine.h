@@ -24,9 +24,10 @@
 //   h values        {binary32 value, 32-bit tag};
 //   stack outputs   {binary32 value, 32-bit tag} (the next layer's input).
 // Where nothing is read (one token's output before an independent next token), each CTA
-// stores a per-CTA "unit done" word instead, and the next unit starts once every CTA's word
-// shows the previous unit. Every exchange buffer is zeroed before each launch; tags are never
-// zero.
+// stores a per-CTA "unit done" word instead; the buffers alternate between units, so unit u
+// of independent tokens with expert rows starts once every CTA's word shows unit u-2 (a
+// router-only launch, and a stack's next token, once it shows unit u-1). Every exchange buffer is zeroed before each launch; tags are
+// never zero.
 #pragma once
 #include <stdint.h>
 
