@@ -1345,10 +1345,9 @@ __device__ __forceinline__ X4 router_x4(const Geo& G, const float* XB, int seg, 
   return X4{(double)v.x, (double)v.y, (double)v.z, (double)v.w};
 }
 
-// four products of one row's float4 group f with x, the weights converted to binary64 (the
+// four products of a float4 group of weights with x, the weights converted to binary64 (the
 // products are exact), accumulated in binary64 onto `acc`
-__device__ __forceinline__ double row_dot4(const float4* ws, int f, const X4& x, double acc) {
-  const float4 wv = ws[f];
+__device__ __forceinline__ double dot4(const float4 wv, const X4& x, double acc) {
   acc = fma((double)wv.x, x.a, acc);
   acc = fma((double)wv.y, x.b, acc);
   acc = fma((double)wv.z, x.c, acc);
@@ -1378,14 +1377,23 @@ __device__ __forceinline__ void router_batch(const Prog& P, const Geo& G, Smem* 
   double v[kRouterBatch];
 #pragma unroll
   for (int r = 0; r < kRouterBatch; ++r) v[r] = 0.0;
+  // every x and weight group of this thread loaded first (clamped to a valid group; the
+  // clamped ones are not used), then the binary64 chains in the same order as one at a time
+  float4 xv[4], wv[4][kRouterBatch];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int f = t + kConsumers * j;
-    if (f < nf) {
-      const X4 x = router_x4(G, XB, 0, f);
+    const int f = min(t + kConsumers * j, nf - 1);
+    xv[j] = reinterpret_cast<const float4*>(XB)[f];
+#pragma unroll
+    for (int r = 0; r < kRouterBatch; ++r) wv[j][r] = ws[r][f];
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (t + kConsumers * j < nf) {
+      const X4 x{(double)xv[j].x, (double)xv[j].y, (double)xv[j].z, (double)xv[j].w};
 #pragma unroll
       for (int r = 0; r < kRouterBatch; ++r)
-        if (r < nrows) v[r] = row_dot4(ws[r], f, x, v[r]);
+        if (r < nrows) v[r] = dot4(wv[j][r], x, v[r]);
     }
   }
   FMOE_MARK_W(u, MK_R_DOT, MK_R_DOT_W);
@@ -1428,7 +1436,7 @@ __device__ __forceinline__ bool router_chunk(const Prog& P, const Geo& G, Smem* 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int f = t + kConsumers * j;
-      if (f < nf) a = row_dot4(ws + (size_t)r * nf, f, router_x4(G, XB, c.seg, f), a);
+      if (f < nf) a = dot4(ws[(size_t)r * nf + f], router_x4(G, XB, c.seg, f), a);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
