@@ -6,7 +6,11 @@ round-robin copies of router / shared expert as bench.py runs it) and prints, fo
 77, the median over units 8..62 of each event's time after the unit's previous-unit-done
 event, in microseconds, with its range. The marks themselves cost a few per cent of a unit.
 
-    python -m bit_dequant_expert_gemv_b200.timeline.timeline [workload]
+With --all-ctas (libfmoe_trace_all.so, every CTA recorded) it prints instead, per CTA, how
+far its unit start lags the median CTA's, the median durations of its phases, and when the
+unit's last router logits were stored relative to the median CTA's start of the top-K.
+
+    python -m bit_dequant_expert_gemv_b200.timeline.timeline [workload] [--all-ctas]
 """
 from __future__ import annotations
 
@@ -21,7 +25,8 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 SO = os.path.join(HERE, "libfmoe_trace.so")
-UNITS, EVENTS = 64, 88          # as in marks.cuh
+SO_ALL = os.path.join(HERE, "libfmoe_trace_all.so")
+UNITS, EVENTS, ALL_CTAS = 64, 88, 148   # as in marks.cuh
 TOKENS = 64
 
 # event ids of engine.cu's MarkEv, as printed
@@ -46,25 +51,71 @@ for k in range(8):
     NAMES[54 + k] = f"K D_{k} done"
 
 
-def build_traced(_build) -> None:
+def build_traced(_build, all_ctas: bool = False) -> str:
     """The engine with the marks force-included; the other sources as in the library."""
+    so = SO_ALL if all_ctas else SO
     srcs = [os.path.join(_build.CSRC, f) for f in _build.SOURCES + _build.HEADERS]
     srcs.append(os.path.join(HERE, "marks.cuh"))
-    if os.path.exists(SO) and os.path.getmtime(SO) >= max(os.path.getmtime(f) for f in srcs):
-        return
+    if os.path.exists(so) and os.path.getmtime(so) >= max(os.path.getmtime(f) for f in srcs):
+        return so
     objs = []
     for src in _build.SOURCES:
-        o = os.path.join(HERE, src + ".o")
+        o = os.path.join(HERE, src + (".all" if all_ctas else "") + ".o")
         cmd = ["nvcc", "-O3", "-std=c++17", *_build.ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
                "-I", _build.INCLUDE, "-I", _build.CSRC]
+        if all_ctas:
+            cmd.append("-DFMOE_TRACE_ALL_CTAS")
         if src == "engine.cu":
             cmd += ["-include", os.path.join(HERE, "marks.cuh")]
         subprocess.run(cmd + ["-c", os.path.join(_build.CSRC, src), "-o", o], check=True)
         objs.append(o)
-    subprocess.run(["nvcc", *_build.ARCH, "-shared", *objs, "-o", SO, "-lcudart"], check=True)
+    subprocess.run(["nvcc", *_build.ARCH, "-shared", *objs, "-o", so, "-lcudart"], check=True)
+    return so
 
 
-def main(wl_name: str = "full_q4") -> None:
+# phases of a unit for the per-CTA view: (name, from event, to event; None = next unit's x)
+PHASES = [("router", 24, 25), ("x digits", 25, 26), ("shared g/u", 26, 27), ("top-K", 3, 4),
+          ("routed g/u 0", 30, 38), ("routed g/u 3", 33, 41), ("shared down", 28, 29),
+          ("down 3", 56, 57), ("outputs", 57, 62), ("unit period", 24, None)]
+
+
+def report_all_ctas(buf, nctas: int) -> None:
+    """Per-CTA phase shifts and durations (medians over units 8..62), in microseconds."""
+    us = lambda a, b: (int(a) - int(b)) / 1000.0  # noqa: E731
+    units = range(8, 62)
+    lag = {c: [] for c in range(nctas)}
+    for u in units:
+        starts = [int(buf[c, u, 24]) for c in range(nctas) if buf[c, u, 24]]
+        med = statistics.median(starts)
+        for c in range(nctas):
+            if buf[c, u, 24]:
+                lag[c].append((int(buf[c, u, 24]) - med) / 1000.0)
+    mean_lag = {c: statistics.mean(v) for c, v in lag.items() if v}
+    order = sorted(mean_lag, key=lambda c: -mean_lag[c])
+    print("unit start after the median CTA's (mean over units 8..61, us):")
+    print("  latest:  " + "  ".join(f"CTA {c} {mean_lag[c]:+.2f}" for c in order[:6]))
+    print("  earliest: " + "  ".join(f"CTA {c} {mean_lag[c]:+.2f}" for c in order[-3:]))
+    print("phase durations (median over units, us): min / median / max over CTAs")
+    for name, a, b in PHASES:
+        per = []
+        for c in range(nctas):
+            v = [us(buf[c, u + 1, 24] if b is None else buf[c, u, b], buf[c, u, a]) for u in units
+                 if buf[c, u, a] and (buf[c, u + 1, 24] if b is None else buf[c, u, b])]
+            if v:
+                per.append(statistics.median(v))
+        if per:
+            print(f"  {name:14s} {min(per):6.2f} {statistics.median(per):6.2f} {max(per):6.2f}")
+    gaps = []
+    for u in units:
+        last_logit = max(int(buf[c, u, 70]) for c in range(nctas))
+        topk_starts = [int(buf[c, u, 3]) for c in range(nctas) if buf[c, u, 3]]
+        if last_logit and topk_starts:
+            gaps.append((last_logit - statistics.median(topk_starts)) / 1000.0)
+    if gaps:
+        print(f"last logits stored, after the median CTA's top-K start: median {statistics.median(gaps):+.2f} us")
+
+
+def main(wl_name: str = "full_q4", all_ctas: bool = False) -> None:
     sys.path.insert(0, ROOT)
     import torch
     import synth
@@ -72,8 +123,7 @@ def main(wl_name: str = "full_q4") -> None:
     from bit_dequant_expert_gemv_b200 import _build
     from bit_dequant_expert_gemv_b200.workload import build_layer, token_inputs_dev
 
-    build_traced(_build)
-    fmoe.LIB = SO
+    fmoe.LIB = build_traced(_build, all_ctas)
     lib = fmoe.lib()
     lib.fmoe_trace_read.argtypes = [C.c_void_p, C.c_size_t]
     wl = synth.WORKLOADS[wl_name]
@@ -101,8 +151,12 @@ def main(wl_name: str = "full_q4") -> None:
     torch.cuda.synchronize()
     print(f"{wl_name}: {a.elapsed_time(b) * 1000 / TOKENS:.2f} us per unit (profiling build)")
     assert fmoe.sync_status() == 0
-    buf = np.zeros((2, UNITS, EVENTS), dtype=np.uint64)
+    nctas = ALL_CTAS if all_ctas else 2
+    buf = np.zeros((nctas, UNITS, EVENTS), dtype=np.uint64)
     assert lib.fmoe_trace_read(buf.ctypes.data, buf.nbytes) == 0
+    if all_ctas:
+        report_all_ctas(buf, min(nctas, int(torch.cuda.get_device_properties(0).multi_processor_count)))
+        return
     for cta in range(2):
         print(f"--- CTA {0 if cta == 0 else 77}: median over units 8..62 of "
               f"(event - 'C prev unit done'), us [min max]")
@@ -119,4 +173,5 @@ def main(wl_name: str = "full_q4") -> None:
 
 
 if __name__ == "__main__":
-    main(*sys.argv[1:2])
+    args = [a for a in sys.argv[1:] if not a.startswith("--")]
+    main(*args[:1], all_ctas="--all-ctas" in sys.argv[1:])
