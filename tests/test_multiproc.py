@@ -64,6 +64,7 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1, r.stdout
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["steps"] == 1 and d["warmup"] == 1  # the untimed warm-up samples are reported
     assert d["config"]["workload"] == "tiny" and d["config"]["parallelism"] == "replicas x2"
     for k in ("cpu_baseline", "e2e"):
         assert k in d
